@@ -1,0 +1,444 @@
+"""Benchmark: the full 32-layer paged decode step at the pages' scale.
+
+Workload (one "step"): 200 concurrent requests, GPT-style 32 layers x 32
+heads x head_dim 128 in fp16 (512 KB of K/V per token), block_size 16,
+context lengths min(2048, 1 + floor(Exponential(mean 500))), every
+sequence's blocks placed at random in one block-id space shared by all
+layers.  Per layer: reshape_and_cache of the step's new token, then paged
+decode attention; the work plan is built once per step and shared by the 32
+layers.  Inputs are synthetic (seeded), the K/V pools are resident in HBM
+and far larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  Metric: KV bytes the attention reads per second
+(GB/s), with decode tokens/s and the HBM-roofline fraction beside it.
+Multi-GPU runs are independent replicas (weak scaling): every rank owns its
+own 200 requests; the only collective is the max-over-ranks of the timing.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+S, LAYERS, H, D, BS = 200, 32, 32, 128, 16
+ELT = 2  # fp16
+WORKLOAD = "full 32-layer decode step: 200 requests, 32 layers x 32 heads x 128 fp16, block 16"
+METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s"
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_478_b200", "csrc", "decode.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_kernel_full_step.md")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kv_bytes(lens):
+    """Algorithmic K/V bytes one layer's decode must read: every cached token,
+    K and V, every head (16 KB per token per layer at 32 x 128 fp16)."""
+    return int(np.sum(lens.astype(np.int64))) * H * D * ELT * 2
+
+
+def algorithmic_bytes_per_launch(lens):
+    """K/V reads plus reading q and writing out (one layer)."""
+    return kv_bytes(lens) + 2 * S * H * D * ELT
+
+
+def decode_source_hash():
+    with open(DECODE_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("decode.cuh sha256[:16]") != decode_source_hash():
+        return None
+    try:
+        return float(vals["dram bytes per launch (read + write)"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---- clocks sampled during the timed region ------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.proc = None
+        self.uuid = uuid
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ---- the CPU oracle as a baseline --------------------------------------------------------
+
+def oracle_sample_case(seed, num_seqs_sample):
+    """The first num_seqs_sample requests of the workload, one layer, on the host."""
+    from paged_kv_cache_478_b200 import synthetic as syn
+
+    lens = syn.full_step_lengths(seed=seed, num_seqs=S)[:num_seqs_sample]
+    return syn.decode_case(seed, lens, H, D, np.float16)
+
+
+def time_oracle(case, reps=1):
+    import oracle
+
+    cores = len(os.sched_getaffinity(0))
+    os.environ["OMP_NUM_THREADS"] = str(cores)
+    kp, vp = case["k_pool"].copy(), case["v_pool"].copy()
+    slots = np.array([oracle.slot_of_c(case["block_tables"][s], int(L) - 1)
+                      for s, L in enumerate(case["context_lens"])], dtype=np.int32)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.reshape_and_cache(case["k_new"], case["v_new"], slots, kp, vp)
+        oracle.decode_attention(case["q"], kp, vp, case["block_tables"], case["context_lens"],
+                                case["scale"], num_threads=cores)
+    dt = (time.perf_counter() - t0) / reps
+    return kv_bytes(case["context_lens"]) / dt / 1e9, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.build()
+    n_sample = 40
+    case = oracle_sample_case(0, n_sample)
+    for _ in range(args.warmup):
+        time_oracle(case)
+    t0 = time.perf_counter()
+    vals = []
+    cores = 1
+    for _ in range(args.steps):
+        v, cores = time_oracle(case)
+        vals.append(v)
+    elapsed = time.perf_counter() - t0
+    value = kv_bytes(case["context_lens"]) * args.steps / elapsed / 1e9
+    sample = (f"one layer of the first {n_sample} of the 200 requests "
+              f"({int(case['context_lens'].sum())} cached tokens, 32 heads x 128 fp16) per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * elapsed / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---- our CUDA path -------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_478_b200 as pa
+    from paged_kv_cache_478_b200 import synthetic as syn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # every rank owns its own 200 requests (weak scaling): seed = rank
+    lens = syn.full_step_lengths(seed=rank, num_seqs=S)
+    tables, nb = syn.full_step_tables(rank, lens)
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    kpools, vpools = [], []
+    for layer in range(LAYERS):
+        kp = torch.empty((nb, H, BS, D), dtype=torch.float16, device=dev)
+        vp = torch.empty_like(kp)
+        syn.fill_normal_device(kp, 1000 * (rank + 1) + 2 * layer)
+        syn.fill_normal_device(vp, 1000 * (rank + 1) + 2 * layer + 1)
+        kpools.append(kp)
+        vpools.append(vp)
+    q = torch.empty((LAYERS, S, H, D), dtype=torch.float16, device=dev)
+    k_new, v_new = torch.empty_like(q), torch.empty_like(q)
+    for t, sd in ((q, 7), (k_new, 8), (v_new, 9)):
+        syn.fill_normal_device(t, 100 * (rank + 1) + sd)
+    out = torch.empty_like(q)
+    bt = torch.from_numpy(tables).to(dev)
+    cl = torch.from_numpy(lens).to(dev)
+    slots = torch.from_numpy(pa.pa_decode_slots(tables, lens)).to(dev)
+    ps = args.partition_size
+    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, ps),
+                     dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    max_parts = math.ceil(tables.shape[1] * BS / (ps or 256))
+    kernels_per_step = 1 + LAYERS * (2 + (1 if max_parts > 1 else 0))
+
+    ev_pairs = []
+
+    def step(record=False):
+        pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=ps)
+        for layer in range(LAYERS):
+            pa.pa_reshape_and_cache(pool, k_new[layer], v_new[layer], slots, kpools[layer],
+                                    vpools[layer])
+            if record:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            pa.pa_decode_attention_planned(pool, q[layer], kpools[layer], vpools[layer], bt, scale,
+                                           out[layer], ws, partition_size=ps)
+            if record:
+                e1.record(stream)
+                ev_pairs.append((e0, e1))
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    assert pa.pa_device_errors() == 0, "device error bits set during warm-up"
+
+    uuid = torch.cuda.get_device_properties(dev).uuid
+    sampler = ClockSampler(f"GPU-{uuid}" if not str(uuid).startswith("GPU-") else str(uuid))
+    sampler.start()
+    time.sleep(0.5)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    errs = pa.pa_device_errors()
+    assert errs == 0, f"device error bits {errs:#x}"
+    decode_ms = [a.elapsed_time(b) for a, b in ev_pairs]
+    decode_avg_ms = float(np.mean(decode_ms))
+
+    ms_per_step = elapsed_ms / args.steps
+    step_kv = kv_bytes(lens) * LAYERS
+    value = step_kv * world / (ms_per_step * 1e-3) / 1e9
+    tokens_per_s = S * world / (ms_per_step * 1e-3)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    per_launch = algorithmic_bytes_per_launch(lens)
+    achieved = per_launch / (decode_avg_ms * 1e-3) / 1e9
+
+    e2e = None if args.no_e2e else run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens,
+                                          ws, ps, world, dev)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        case = oracle_sample_case(0, 40)
+        v, cores = time_oracle(case)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"one layer of the first 40 of the 200 requests "
+                         f"({int(case['context_lens'].sum())} cached tokens), fp64 C oracle, "
+                         f"OpenMP over (sequence, head)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "num_seqs": S, "layers": LAYERS, "heads": H,
+                       "head_dim": D, "block_size": BS, "cached_tokens": int(lens.sum()),
+                       "pool_blocks": nb, "partition_size": ps or 256,
+                       "kv_bytes_per_step": step_kv, "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"replicas x{world}"},
+            "decode_tokens_per_s": round(tokens_per_s, 1),
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": committed_traffic(),
+                         "peak_kind": peak_kind,
+                         "kernel": "paged_decode_kernel + merge (events bracket one planned call)",
+                         "bytes_per_launch": per_launch,
+                         "avg_launch_ms": round(decode_avg_ms, 5)},
+            "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, dev):
+    """The same step through the same calls, with the step's inputs (q, k_new,
+    v_new of every layer, block tables, lengths, slots) copied from pinned host
+    memory and the outputs read back every step.  Copies run on a side stream
+    so layer l+1's inputs cross PCIe while layer l computes."""
+    import torch.distributed as dist
+
+    main = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    rng = np.random.default_rng(11)
+    h_q = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
+    h_k = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
+    h_v = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
+    h_out = torch.empty((LAYERS, S, H, D), dtype=torch.float16).pin_memory()
+    h_bt = torch.from_numpy(tables).pin_memory()
+    h_cl = torch.from_numpy(lens).pin_memory()
+    h_slots = torch.empty(S, dtype=torch.int32).pin_memory()
+    d_q = torch.empty((LAYERS, S, H, D), dtype=torch.float16, device=dev)
+    d_k, d_v, d_out = torch.empty_like(d_q), torch.empty_like(d_q), torch.empty_like(d_q)
+    d_bt = torch.empty_like(h_bt, device=dev)
+    d_cl = torch.empty_like(h_cl, device=dev)
+    d_slots = torch.empty(S, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    h2d = 3 * d_q.numel() * 2 + h_bt.numel() * 4 + h_cl.numel() * 4 + S * 4
+    d2h = d_out.numel() * 2
+
+    def step():
+        h_slots.copy_(torch.from_numpy(pa.pa_decode_slots(tables, lens)))  # host scheduler work
+        in_ready = []
+        with torch.cuda.stream(copy):
+            d_bt.copy_(h_bt, non_blocking=True)
+            d_cl.copy_(h_cl, non_blocking=True)
+            d_slots.copy_(h_slots, non_blocking=True)
+            for layer in range(LAYERS):
+                d_q[layer].copy_(h_q[layer], non_blocking=True)
+                d_k[layer].copy_(h_k[layer], non_blocking=True)
+                d_v[layer].copy_(h_v[layer], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy)
+                in_ready.append(ev)
+        main.wait_event(in_ready[0])
+        pa.pa_decode_plan(pool, d_cl, tables.shape[1], ws, partition_size=ps)
+        for layer in range(LAYERS):
+            main.wait_event(in_ready[layer])
+            pa.pa_reshape_and_cache(pool, d_k[layer], d_v[layer], d_slots, kpools[layer],
+                                    vpools[layer])
+            pa.pa_decode_attention_planned(pool, d_q[layer], kpools[layer], vpools[layer], d_bt,
+                                           scale, d_out[layer], ws, partition_size=ps)
+            done = torch.cuda.Event()
+            done.record(main)
+            copy.wait_event(done)
+            with torch.cuda.stream(copy):
+                h_out[layer].copy_(d_out[layer], non_blocking=True)
+        main.wait_stream(copy)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(main)
+    for _ in range(args.steps):
+        step()
+    t1.record(main)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert torch.isfinite(h_out.float()).all()
+    value = kv_bytes(lens) * LAYERS * world / (ms * 1e-3) / 1e9
+    return {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
+            "decode_tokens_per_s": round(S * world / (ms * 1e-3), 1)}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

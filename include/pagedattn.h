@@ -1,0 +1,256 @@
+/*
+ * pagedattn.h: C ABI of the paged decode-attention library (libpagedattn.so).
+ *
+ * What it computes (sources are web pages on PagedAttention):
+ *   - "Atención paginada en modelos de lenguaje grandes (LLM)" (7minutos.es),
+ *     section 2: the KV cache lives in a flat pool of equal physical pages of
+ *     16 tokens; a request's block_table maps logical page i to a physical
+ *     page id, and a new page is claimed only when the token count crosses a
+ *     page boundary.  Section 3: pages are reference-counted and shared by
+ *     requests with a common prefix; share() raises the count, cow_copy()
+ *     gives a writer a private copy and lowers the original's count.
+ *   - "PagedAttention" (e-fortepiano.pl wiki mirror), "Descripció": logical
+ *     blocks need not be physically contiguous; "Formulació matemàtica": the
+ *     attention of one query token is computed block by block over the KV
+ *     blocks and equals the ordinary softmax(q.K^T * scale).V.
+ *
+ * Data layout (all device buffers are owned by the caller):
+ *   k_pool, v_pool   [num_blocks][heads][block_size][head_dim], dtype elements,
+ *                    16-byte aligned base.  Physical slot of a token =
+ *                    block_id * block_size + in-block offset.
+ *   q, out           [num_seqs][heads][head_dim], same dtype as the pool.
+ *   k_new, v_new     [num_tokens][heads][head_dim], same dtype as the pool.
+ *   block_tables     int32 [num_seqs][max_blocks_per_seq]; entries past a
+ *                    sequence's last block are never read.
+ *   context_lens     int32 [num_seqs]: tokens cached per sequence, counting
+ *                    the token appended this step.
+ *   slot_mapping     int32 [num_tokens]; a negative slot is skipped (padding).
+ *   pairs            int32 [num_pairs][2] = (src_block, dst_block).
+ *
+ * Errors: every call returns a pa_status; PA_OK means the arguments passed
+ * host-side validation and the kernels were enqueued on `stream` (a
+ * cudaStream_t; NULL is the legacy default stream).  Launches are
+ * asynchronous.  Values that only the device sees (block ids, slots, context
+ * lengths) are bounds-checked in the kernels: a bad value is skipped or
+ * clamped, never dereferenced, and raises a bit in a per-device error word
+ * that pa_device_errors() returns and clears.  pa_last_error() gives a
+ * message for the last failing call on the calling thread.
+ *
+ * Supported: block_size 16; head_dim 64 or 128; dtype fp32, fp16, bf16.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
+  PA_ERR_UNSUPPORTED = 2,   /* dtype / head_dim / block_size not built */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime call failed; see pa_last_error() */
+  PA_ERR_OUT_OF_BOUNDS = 4, /* device-side bounds check fired */
+  PA_ERR_NO_FREE_BLOCKS = 5,/* block manager: pool exhausted */
+  PA_ERR_WORKSPACE = 6,     /* workspace missing or too small */
+  PA_ERR_TIMEOUT = 7        /* a device-side wait gave up */
+} pa_status;
+
+/* Bits of the device error word (pa_device_errors). */
+#define PA_DEVERR_BLOCK_ID 0x1u    /* block table entry outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 0x2u        /* slot outside [0, num_blocks * block_size) */
+#define PA_DEVERR_CONTEXT_LEN 0x4u /* context_len < 0 or above the table / max bound */
+#define PA_DEVERR_PAIR 0x8u        /* copy_blocks pair outside the pool */
+#define PA_DEVERR_TIMEOUT 0x10u    /* an mbarrier wait ran past its limit */
+
+/* Plain value descriptor of one K or V pool (the two share it). */
+typedef struct pa_pool {
+  int64_t num_blocks;
+  int32_t block_size;
+  int32_t heads;
+  int32_t head_dim;
+  int32_t dtype;       /* pa_dtype */
+  int32_t elem_bytes;
+  int32_t reserved;
+  int64_t token_stride; /* elements between consecutive slots of a block: head_dim */
+  int64_t head_stride;  /* elements between heads of a block: block_size * head_dim */
+  int64_t block_stride; /* elements between blocks: heads * block_size * head_dim */
+  int64_t bytes_per_pool; /* bytes of ONE of k_pool / v_pool */
+} pa_pool;
+
+/*
+ * Describe a pool (section 2 of the 7minutos.es article: a flat array of
+ * equal pages).  Allocates nothing; fills *out.  num_blocks * block_size must
+ * stay below 2^31 so that slots fit int32.
+ * Errors: PA_ERR_INVALID_ARG (non-positive sizes, null out, slot overflow),
+ *         PA_ERR_UNSUPPORTED (block_size != 16, head_dim not 64/128, dtype).
+ */
+pa_status pa_pool_create(int64_t num_blocks, int32_t block_size, int32_t heads,
+                         int32_t head_dim, int32_t dtype, pa_pool* out);
+
+/*
+ * Write each new token's K and V rows into the slot slot_mapping names:
+ * k_pool[slot / bs][h][slot % bs][:] = k_new[t][h][:] for every head, the
+ * same for V (7minutos.es section 2: the new token goes into the tail page).
+ * Bit copy.  A negative slot is skipped; a slot >= num_blocks * block_size
+ * sets PA_DEVERR_SLOT and is skipped.  num_tokens == 0 is a no-op.
+ */
+pa_status pa_reshape_and_cache(const pa_pool* pool, const void* k_new, const void* v_new,
+                               const int32_t* slot_mapping, int32_t num_tokens, void* k_pool,
+                               void* v_pool, void* stream);
+
+/*
+ * Bytes of device workspace pa_decode_attention needs for these sizes
+ * (work plan + split-K partial results).  partition_size 0 = the default.
+ * max_context_len 0 = max_blocks_per_seq * block_size.
+ */
+pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
+                                    int32_t max_blocks_per_seq, int32_t max_context_len,
+                                    int32_t partition_size, size_t* bytes);
+
+/*
+ * Single-query decode attention over the paged cache ("PagedAttention" wiki
+ * mirror, "Formulació matemàtica"): for every sequence s and head h,
+ *   out[s][h] = sum_t softmax_t(scale * q[s][h] . K_t) V_t,  t < context_lens[s],
+ * with K_t, V_t read through block_tables[s].  fp32 accumulation, online
+ * softmax; the result is rounded to the pool dtype.  A sequence of length 0
+ * gets zeros.
+ * Long contexts are split into partitions of partition_size tokens (a
+ * multiple of 16; 0 = default 256) whose partial results are merged by
+ * log-sum-exp in a second kernel.  The work order is planned on the device
+ * from context_lens (longest partitions first).
+ * max_context_len bounds every context_lens[s] (0 = max_blocks_per_seq *
+ * block_size); a length above it or above the table width sets
+ * PA_DEVERR_CONTEXT_LEN and is clamped.  Block ids outside the pool set
+ * PA_DEVERR_BLOCK_ID and are replaced by block 0.
+ * workspace: device buffer of at least pa_decode_workspace_bytes(); its
+ * contents on entry do not matter.  Calls that share a workspace must be
+ * ordered on one stream.
+ * Errors: PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA.
+ */
+pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_pool,
+                              const void* v_pool, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t max_context_len, float scale, void* out,
+                              void* workspace, size_t workspace_bytes, int32_t partition_size,
+                              void* stream);
+
+/*
+ * The two halves of pa_decode_attention, for callers that run many layers
+ * over the same context lengths in one step (every layer of a model shares
+ * the step's block tables and lengths):
+ *   pa_decode_plan writes the work plan (clamped lengths, partitions per
+ *   sequence, work items ordered longest first) into the workspace;
+ *   pa_decode_attention_planned runs the partition and merge kernels from it.
+ * A plan stays valid for any number of planned calls with the same pool
+ * geometry (heads, head_dim, dtype), num_seqs, max_blocks_per_seq,
+ * max_context_len and partition_size, issued in stream order on the same
+ * workspace; each planned call leaves the plan ready for the next.
+ */
+pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32_t num_seqs,
+                         int32_t max_blocks_per_seq, int32_t max_context_len,
+                         int32_t partition_size, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const void* k_pool,
+                                      const void* v_pool, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, int32_t num_seqs,
+                                      int32_t max_context_len, float scale, void* out,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t partition_size, void* stream);
+
+/*
+ * Block-granular copy-on-write, device half ("PagedAttention" wiki mirror,
+ * "Descripció"; 7minutos.es section 3, cow_copy): for each (src, dst) row of
+ * pairs (device int32 [num_pairs][2]) copy the whole physical block, every
+ * head and slot, of K and of V.  Bit copy.  No dst may be another pair's src
+ * or dst (the block manager hands out fresh destinations).  Ids outside the
+ * pool set PA_DEVERR_PAIR and the pair is skipped.
+ */
+pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,
+                         int32_t num_pairs, void* stream);
+
+/*
+ * Synchronise `stream`, then return in *flags the PA_DEVERR_* bits raised on
+ * the current device since the last call, and clear them.  Returns
+ * PA_ERR_OUT_OF_BOUNDS / PA_ERR_TIMEOUT when a bit is set, else PA_OK.
+ */
+pa_status pa_device_errors(void* stream, uint32_t* flags);
+
+/*
+ * Self-test of the device-side wait limit: launches one warp that waits on
+ * an mbarrier nothing will complete, so the bounded wait used by the decode
+ * pipeline runs out (about one second), raises PA_DEVERR_TIMEOUT and returns.
+ * Nothing faults and the context stays usable; read the bit with
+ * pa_device_errors().  No counterpart on the pages: it exists to test the
+ * failure path without a GPU fault.
+ */
+pa_status pa_selftest_wait_timeout(void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+/* Fixed name of a status code. */
+const char* pa_status_string(int32_t status);
+
+/* ---- host block manager (reference counts and free list stay on the host) ----
+ * 7minutos.es, sections 2 and 3: a pool of pages with a free list and a
+ * reference count per page; a page returns to the free list as soon as its
+ * count reaches zero.  The lowest free id is handed out first.  Not
+ * thread-safe: one manager per thread, or lock around it. */
+typedef struct pa_allocator pa_allocator;
+
+pa_status pa_alloc_create(int64_t num_blocks, pa_allocator** out);
+void pa_alloc_destroy(pa_allocator* a);
+/* Take the lowest free block (refcount becomes 1); PA_ERR_NO_FREE_BLOCKS if none. */
+pa_status pa_alloc_block(pa_allocator* a, int32_t* block_id);
+/* share(): one more holder of a live block; allocates nothing. */
+pa_status pa_share_block(pa_allocator* a, int32_t block_id);
+/* Drop one holder; at zero the block goes back to the free list. */
+pa_status pa_free_block(pa_allocator* a, int32_t block_id);
+/* cow_copy(): allocate a private block for one holder of a live block and
+ * drop that holder's reference to the original.  The caller copies the data
+ * (pa_copy_blocks). */
+pa_status pa_cow_block(pa_allocator* a, int32_t block_id, int32_t* new_block_id);
+pa_status pa_refcount(const pa_allocator* a, int32_t block_id, int32_t* refcount);
+int64_t pa_num_free(const pa_allocator* a);
+
+/*
+ * Append num_new tokens to one sequence (generate_token() of section 2).
+ * block_table holds ceil(*context_len / block_size) live block ids and has
+ * room for max_blocks.  For each new token at position p: a fresh block is
+ * taken when p is a multiple of block_size; otherwise, if the tail block is
+ * shared (refcount > 1), it is copied on write (section 3) and the
+ * (src, dst) pair is appended to cow_pairs (room for num_new pairs).
+ * slots[i] receives the physical slot of the i-th new token.  On error the
+ * tokens appended before it stay appended (*context_len and *num_cow say how
+ * far it got).
+ */
+pa_status pa_append_tokens(pa_allocator* a, int32_t block_size, int32_t* block_table,
+                           int32_t max_blocks, int32_t* context_len, int32_t num_new,
+                           int32_t* slots, int32_t* cow_pairs, int32_t* num_cow);
+
+/* Give dst_table the same blocks as src_table (prefix sharing: one share()
+ * per block). */
+pa_status pa_fork_table(pa_allocator* a, const int32_t* src_table, int32_t num_blocks,
+                        int32_t* dst_table);
+
+/* Drop the sequence's reference to each of its blocks (request finished). */
+pa_status pa_release_table(pa_allocator* a, const int32_t* block_table, int32_t num_blocks);
+
+/* Host helper for tables built elsewhere: slot of the last token of each
+ * sequence, block_tables[s][(L-1)/bs] * bs + (L-1) % bs, or -1 when L == 0.
+ * All pointers are host memory. */
+pa_status pa_decode_slots(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
+                          int32_t* slots);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,414 @@
+// Paged decode attention for sm_100a: work plan, partition kernel, split-K merge.
+//
+// The method: "PagedAttention" (e-fortepiano.pl wiki mirror), "Formulació
+// matemàtica" -- the attention of one query token, computed block by block
+// over KV blocks reached through the sequence's block table, equals the
+// ordinary softmax(q.K^T * scale).V over the cached tokens.  Block table and
+// 16-token pages: "Atención paginada en modelos de lenguaje grandes (LLM)"
+// (7minutos.es), section 2.
+//
+// Design (ours; the pages give no kernel):
+//   * The unit of work is (sequence s, partition p of partition_size tokens,
+//     group g of WARPS heads).  One warp owns one head of the group, so the
+//     warps of a CTA share the block-table slice and read adjacent 4 KB tiles
+//     of the same physical block.
+//   * Each warp runs its own NSTAGE-deep ring of shared-memory stages.  Lane
+//     0 issues two 1-D bulk copies per stage (the K and V tiles of one
+//     (block, head), contiguous in the [block][head][slot][dim] layout) that
+//     complete on that stage's mbarrier; no multicast, no tensor map.
+//   * q.k: lane l reads 16-byte chunks l, l+32, ... of the tile from shared
+//     memory (512 contiguous bytes per warp instruction, conflict free); a
+//     transpose-reduce over the lanes of a row leaves every lane with one
+//     token's score in NCH shuffles instead of NCH*log2(LPR).
+//   * fp32 online softmax in the log2 domain (q is pre-scaled by
+//     scale*log2(e)); P.V accumulates in fp32 registers.
+//   * Work items are handed out by an atomic counter in the workspace, in the
+//     order a one-CTA plan kernel wrote: full partitions first, then the
+//     ragged last partitions by decreasing size, so the tail of the grid is
+//     made of the smallest items.
+//   * Sequences with more than one partition write (m, l, unnormalised acc)
+//     per partition; the merge kernel combines them by log-sum-exp in
+//     partition order.  No atomics touch values, so results are bit-stable
+//     run to run and independent of where the blocks sit in the pool.
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+
+#include "device_utils.cuh"
+#include "pagedattn.h"
+
+namespace pa {
+
+constexpr int kBlock = 16;  // tokens per physical block
+
+struct PlanHeader {
+  int32_t num_pairs;     // (sequence, partition) pairs
+  int32_t num_items;     // num_pairs * head_groups
+  int32_t work_counter;  // next item index to hand out
+  int32_t done_counter;  // CTAs that have left the work loop
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_pool;
+  const void* v_pool;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  void* out;
+  PlanHeader* plan;
+  int32_t* lens;    // [S] clamped context lengths
+  int32_t* nparts;  // [S] partitions per sequence (>= 1)
+  int2* pairs;      // [S * max_parts] work pairs (s, p)
+  float2* part_ml;  // [S][H][max_parts] (running max in log2 units, sum of weights)
+  float* part_acc;  // [S][H][max_parts][D] unnormalised partial outputs
+  uint32_t* err;
+  int64_t num_blocks;
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+  int32_t heads;
+  int32_t head_groups;
+  int32_t partition_size;
+  int32_t max_parts;
+  int32_t max_context_len;
+  float scale_log2;  // scale * log2(e)
+};
+
+// ---- plan: one CTA orders the work ------------------------------------------------
+
+__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
+  extern __shared__ int32_t bucket[];  // [nb + 1]: index 0 = empty sequences
+  __shared__ int32_t n_full;
+  const int PS = a.partition_size;
+  const int nb = PS / kBlock;
+  for (int i = threadIdx.x; i <= nb; i += blockDim.x) bucket[i] = 0;
+  if (threadIdx.x == 0) n_full = 0;
+  __syncthreads();
+  const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
+  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+    int L = a.context_lens[s];
+    if (L < 0 || L > cap) {
+      atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+      L = L < 0 ? 0 : cap;
+    }
+    a.lens[s] = L;
+    const int full = L / PS, rem = L % PS;
+    a.nparts[s] = max(1, full + (rem > 0 ? 1 : 0));
+    if (full > 0) {
+      const int pos = atomicAdd(&n_full, full);
+      for (int p = 0; p < full; ++p) a.pairs[pos + p] = make_int2(s, p);
+    }
+    if (L == 0 || rem > 0) atomicAdd(&bucket[L == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = n_full;
+    for (int b = nb; b >= 0; --b) {  // biggest remainders first, empty sequences last
+      const int c = bucket[b];
+      bucket[b] = run;
+      run += c;
+    }
+    a.plan->num_pairs = run;
+    a.plan->num_items = run * a.head_groups;
+    a.plan->work_counter = 0;
+    a.plan->done_counter = 0;
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+    const int L = a.lens[s];
+    const int rem = L % PS;
+    if (L == 0 || rem > 0) {
+      const int pos = atomicAdd(&bucket[L == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
+      a.pairs[pos] = make_int2(s, L / PS);
+    }
+  }
+}
+
+// ---- transpose-reduce of NCH partial dot products over LPR lanes --------------------
+// Step with xor-mask M halves the values a lane carries: the lane keeps one
+// half and adds its partner's copy of that half.  After log2(NCH) steps one
+// value is left, summed over NCH lanes; a last xor-1 step completes the row.
+
+template <int M, int N>
+__device__ __forceinline__ void halve(float* v, int lane) {
+  if constexpr (M >= 2) {
+    const bool upper = (lane & M) != 0;
+#pragma unroll
+    for (int k = 0; k < N / 2; ++k) {
+      const float send = upper ? v[k] : v[k + N / 2];
+      const float keep = upper ? v[k + N / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(kFullMask, send, M);
+    }
+    halve<M / 2, N / 2>(v, lane);
+  }
+}
+
+// ---- the partition kernel -----------------------------------------------------------
+
+template <typename T, int D, int WARPS, int NSTAGE>
+struct DecodeConfig {
+  static constexpr int VEC = Chunk<T>::N;      // elements per 16-byte chunk
+  static constexpr int CPR = D / VEC;          // chunks (= lanes) per token row
+  static constexpr int RPI = 32 / CPR;         // rows covered by one warp-wide load
+  static constexpr int NCH = kBlock / RPI;     // chunks per lane per tile
+  static constexpr int TILE = kBlock * D * (int)sizeof(T);  // one (block, head) tile
+  static constexpr int STAGE_BYTES = 2 * TILE;              // K tile + V tile
+  static constexpr int THREADS = WARPS * 32;
+  static_assert(CPR >= 2 && CPR <= 32 && 32 % CPR == 0, "head_dim / dtype not supported");
+  static_assert(NCH * 2 == CPR, "lane mapping");
+  static size_t smem_bytes(int partition_size) {
+    return (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
+           (size_t)(partition_size / kBlock) * 4;
+  }
+};
+
+template <typename T, int D, int WARPS, int NSTAGE>
+__global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) {
+  using Cfg = DecodeConfig<T, D, WARPS, NSTAGE>;
+  using C = Chunk<T>;
+  constexpr int VEC = Cfg::VEC, CPR = Cfg::CPR, RPI = Cfg::RPI, NCH = Cfg::NCH;
+  constexpr int TILE = Cfg::TILE;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * NSTAGE * Cfg::STAGE_BYTES);
+  int32_t* tbl = reinterpret_cast<int32_t*>(bars + WARPS * NSTAGE);
+  __shared__ int32_t s_item;
+  __shared__ int32_t s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int H = a.heads;
+  const int PS = a.partition_size;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    mbar_init_fence();
+    s_abort = 0;
+  }
+  int32_t next = 0;
+  if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
+  const int32_t num_items = a.plan->num_items;
+  __syncthreads();
+
+  uint32_t fills = 0;  // stage fills this warp has consumed so far (drives ring slot + parity)
+  uint8_t* my_stages = stages + warp * NSTAGE * Cfg::STAGE_BYTES;
+  uint64_t* my_bars = bars + warp * NSTAGE;
+
+  for (;;) {
+    if (threadIdx.x == 0) {
+      s_item = next;
+      if (next < num_items) next = atomicAdd(&a.plan->work_counter, 1);  // prefetch the next index
+    }
+    __syncthreads();
+    const int item = s_item;
+    if (item >= num_items || s_abort) break;
+
+    const int2 pr = a.pairs[item / a.head_groups];
+    const int g = item % a.head_groups;
+    const int s = pr.x, p = pr.y;
+    const int L = a.lens[s];
+    const bool split = a.nparts[s] > 1;
+    const int tok0 = p * PS;
+    const int ntok = max(0, min(L, tok0 + PS) - tok0);
+    const int nblk = (ntok + kBlock - 1) / kBlock;
+    const int blk0 = tok0 / kBlock;
+
+    // block-table slice of this partition, bounds-checked once
+    for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
+      int32_t b = a.block_tables[(int64_t)s * a.max_blocks_per_seq + blk0 + i];
+      if (b < 0 || b >= a.num_blocks) {
+        atomicOr(a.err, PA_DEVERR_BLOCK_ID);
+        b = 0;
+      }
+      tbl[i] = b;
+    }
+    __syncthreads();
+
+    const int h = g * WARPS + warp;
+    if (h < H) {
+      const int c = lane % CPR;  // this lane's chunk within a token row
+      float qf[VEC];
+      {
+        const uint4 u =
+            reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((int64_t)s * H + h) * D)[c];
+        C::to_float(u, qf);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) qf[e] *= a.scale_log2;
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+      float acc[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+
+      const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)h * TILE;
+      const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)h * TILE;
+      const int64_t block_bytes = (int64_t)H * TILE;
+      auto issue = [&](uint32_t k, int bi) {
+        const int st = k % NSTAGE;
+        const uint32_t bar = smem_addr(&my_bars[st]);
+        uint8_t* dst = my_stages + st * Cfg::STAGE_BYTES;
+        const int64_t off = (int64_t)tbl[bi] * block_bytes;
+        mbar_arrive_expect_tx(bar, 2 * TILE);
+        bulk_copy_g2s(smem_addr(dst), kbase + off, TILE, bar);
+        bulk_copy_g2s(smem_addr(dst + TILE), vbase + off, TILE, bar);
+      };
+
+      const uint32_t k0 = fills;
+      if (lane == 0) {
+        fence_proxy_async_shared();  // the previous item's reads of these stages are done
+        for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
+      }
+      // rows this lane reads: r_j = lane / CPR + RPI * j; score row after the reduce:
+      const int my_row = lane / CPR + RPI * ((lane % CPR) >> 1);
+      bool ok = true;
+      int i = 0;
+      for (; i < nblk; ++i) {
+        const uint32_t k = k0 + i;
+        const int st = k % NSTAGE;
+        const bool landed = mbar_wait_bounded(smem_addr(&my_bars[st]), (k / NSTAGE) & 1u);
+        if (!__all_sync(kFullMask, landed)) {
+          ok = false;
+          break;
+        }
+        const uint4* kt = reinterpret_cast<const uint4*>(my_stages + st * Cfg::STAGE_BYTES);
+        const uint4* vt = kt + TILE / 16;
+        const int valid = min(kBlock, ntok - i * kBlock);
+
+        float part[NCH];
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          float kf[VEC];
+          C::to_float(kt[lane + 32 * j], kf);
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) d = fmaf(qf[e], kf[e], d);
+          part[j] = d;
+        }
+        halve<CPR / 2, NCH>(part, lane);
+        float sc = part[0] + __shfl_xor_sync(kFullMask, part[0], 1);
+        if (my_row >= valid) sc = -INFINITY;
+
+        float bmax = sc;
+#pragma unroll
+        for (int m = 2; m < 32; m <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFullMask, bmax, m));
+        const float m_new = fmaxf(m_run, bmax);
+        const float alpha = exp2f(m_run - m_new);
+        const float pw = exp2f(sc - m_new);
+        float bsum = pw;
+#pragma unroll
+        for (int m = 2; m < 32; m <<= 1) bsum += __shfl_xor_sync(kFullMask, bsum, m);
+        l_run = fmaf(l_run, alpha, bsum);
+        m_run = m_new;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] *= alpha;
+
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          const float pj = __shfl_sync(kFullMask, pw, (lane / CPR) * CPR + 2 * j);
+          float vf[VEC];
+          C::to_float(vt[lane + 32 * j], vf);
+          if (valid < kBlock && lane / CPR + RPI * j >= valid) continue;  // slot past the end
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pj, vf[e], acc[e]);
+        }
+        __syncwarp();
+        if (lane == 0 && i + NSTAGE < nblk) {
+          fence_proxy_async_shared();
+          issue(k + NSTAGE, i + NSTAGE);
+        }
+      }
+      if (!ok) {
+        // give up on this item: report, let the copies already issued land, stop the CTA
+        if (lane == 0) {
+          atomicOr(a.err, PA_DEVERR_TIMEOUT);
+          s_abort = 1;
+        }
+        const int issued = min(nblk, i + NSTAGE);
+        for (int j = i; j < issued; ++j) {
+          const uint32_t k = k0 + j;
+          mbar_wait_bounded(smem_addr(&my_bars[k % NSTAGE]), (k / NSTAGE) & 1u);
+        }
+      } else {
+        fills = k0 + nblk;
+        // combine the RPI lanes that hold the same chunk (different rows)
+#pragma unroll
+        for (int m = CPR; m < 32; m <<= 1) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(kFullMask, acc[e], m);
+        }
+        if (lane < CPR) {
+          const int64_t sh = (int64_t)s * H + h;
+          if (!split) {
+            float o[VEC];
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) o[e] = l_run > 0.f ? acc[e] * inv : 0.f;
+            reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D)[c] = C::from_float(o);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.part_acc + (sh * a.max_parts + p) * D + c * VEC);
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+              dst[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            if (lane == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // the last CTA out re-arms the queue so the plan can be reused
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int done = atomicAdd(&a.plan->done_counter, 1);
+    if (done == (int)gridDim.x - 1) {
+      a.plan->work_counter = 0;
+      a.plan->done_counter = 0;
+      __threadfence();
+    }
+  }
+}
+
+// ---- split-K merge: one warp per (sequence, head) -----------------------------------
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) paged_decode_merge_kernel(DecodeArgs a) {
+  using C = Chunk<T>;
+  constexpr int VEC = C::N;
+  constexpr int CPR = D / VEC;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t sh = (int64_t)blockIdx.x * 4 + warp;
+  if (sh >= (int64_t)a.num_seqs * a.heads) return;
+  const int s = (int)(sh / a.heads);
+  const int np = a.nparts[s];
+  if (np <= 1 || lane >= CPR) return;
+  const float2* ml = a.part_ml + sh * a.max_parts;
+  float M = -INFINITY;
+  for (int p = 0; p < np; ++p) M = fmaxf(M, ml[p].x);
+  float den = 0.f;
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  const float* base = a.part_acc + sh * a.max_parts * D + lane * VEC;
+  for (int p = 0; p < np; ++p) {
+    const float2 v = ml[p];
+    const float w = exp2f(v.x - M);
+    den = fmaf(v.y, w, den);
+    const float4* src = reinterpret_cast<const float4*>(base + (int64_t)p * D);
+#pragma unroll
+    for (int e = 0; e < VEC; e += 4) {
+      const float4 x = src[e / 4];
+      acc[e] = fmaf(w, x.x, acc[e]);
+      acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
+      acc[e + 2] = fmaf(w, x.z, acc[e + 2]);
+      acc[e + 3] = fmaf(w, x.w, acc[e + 3]);
+    }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] *= inv;
+  reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D)[lane] = C::from_float(acc);
+}
+
+}  // namespace pa

@@ -1,0 +1,426 @@
+// C ABI of libpagedattn.so: host-side validation, per-device set-up and
+// kernel launches.  Declarations and argument contracts: include/pagedattn.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "cache_ops.cuh"
+#include "decode.cuh"
+#include "pagedattn.h"
+#include "status.h"
+
+namespace pa {
+
+// Per-device error word raised by the kernels (PA_DEVERR_* bits).
+__device__ uint32_t g_device_errors;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDecodeWarps = 4;   // heads per CTA (one warp each)
+constexpr int kDecodeStages = 3;  // per-warp ring depth
+constexpr int kDefaultPartition = 256;
+constexpr int kMaxPartition = 4096;
+
+struct DeviceState {
+  bool ready = false;
+  uint32_t* err = nullptr;  // device address of g_device_errors
+  int num_sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  char buf[256];
+  std::snprintf(buf, sizeof buf, "%s: %s", what, cudaGetErrorString(e));
+  return fail(PA_ERR_CUDA, buf);
+}
+
+template <typename T, int D>
+using DecodeKernelCfg = DecodeConfig<T, D, kDecodeWarps, kDecodeStages>;
+
+template <typename T, int D>
+cudaError_t set_decode_attrs() {
+  const size_t smem = DecodeKernelCfg<T, D>::smem_bytes(kMaxPartition);
+  return cudaFuncSetAttribute(paged_decode_kernel<T, D, kDecodeWarps, kDecodeStages>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+// Once per device, with that device current: resolve the error word's device
+// address and raise the shared-memory limit of the decode kernels.
+pa_status device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "device index out of range");
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_errors);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_device_errors)");
+    st.err = static_cast<uint32_t*>(p);
+    e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cudaError_t attrs[] = {set_decode_attrs<float, 64>(),          set_decode_attrs<float, 128>(),
+                           set_decode_attrs<__half, 64>(),         set_decode_attrs<__half, 128>(),
+                           set_decode_attrs<__nv_bfloat16, 64>(), set_decode_attrs<__nv_bfloat16, 128>()};
+    for (cudaError_t a : attrs)
+      if (a != cudaSuccess) return cuda_fail(a, "cudaFuncSetAttribute");
+    st.ready = true;
+  }
+  *out = &st;
+  return PA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status check_pool(const pa_pool* pool) {
+  if (!pool) return fail(PA_ERR_INVALID_ARG, "pool descriptor is null");
+  if (pool->block_size != kBlock) return fail(PA_ERR_UNSUPPORTED, "block_size must be 16");
+  if (pool->head_dim != 64 && pool->head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (pool->dtype < PA_F32 || pool->dtype > PA_BF16) return fail(PA_ERR_UNSUPPORTED, "unknown dtype");
+  if (pool->num_blocks <= 0 || pool->heads <= 0) return fail(PA_ERR_INVALID_ARG, "empty pool");
+  if (pool->num_blocks * pool->block_size > INT32_MAX)
+    return fail(PA_ERR_INVALID_ARG, "num_blocks * block_size must fit int32");
+  return PA_OK;
+}
+
+struct WorkspaceLayout {
+  size_t header = 0, lens = 0, nparts = 0, pairs = 0, part_ml = 0, part_acc = 0, total = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D) {
+  WorkspaceLayout w;
+  size_t off = 0;
+  w.header = off;
+  off = align256(off + sizeof(PlanHeader));
+  w.lens = off;
+  off = align256(off + S * 4);
+  w.nparts = off;
+  off = align256(off + S * 4);
+  w.pairs = off;
+  off = align256(off + S * max_parts * 8);
+  w.part_ml = off;
+  off = align256(off + S * H * max_parts * 8);
+  w.part_acc = off;
+  off = align256(off + S * H * max_parts * D * 4);
+  w.total = off;
+  return w;
+}
+
+int resolve_partition(int32_t partition_size) {
+  return partition_size == 0 ? kDefaultPartition : partition_size;
+}
+
+int resolve_max_context(const pa_pool* pool, int32_t max_blocks_per_seq, int32_t max_context_len) {
+  const int64_t cap = (int64_t)max_blocks_per_seq * pool->block_size;
+  const int64_t m = max_context_len == 0 ? cap : std::min<int64_t>(cap, max_context_len);
+  return (int)std::min<int64_t>(m, INT32_MAX);
+}
+
+template <typename T, int D>
+cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
+  using Cfg = DecodeKernelCfg<T, D>;
+  auto kernel = paged_decode_kernel<T, D, kDecodeWarps, kDecodeStages>;
+  const size_t smem = Cfg::smem_bytes(a.partition_size);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Cfg::THREADS, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = std::max(per_sm, 1);
+  const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
+  kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t pairs = (int64_t)a.num_seqs * a.heads;
+  if (a.max_parts > 1) {
+    paged_decode_merge_kernel<T, D><<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+// One warp waits on a barrier that expects two arrivals but gets one.
+__global__ void wait_timeout_selftest_kernel(uint32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 2);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bar)) : "memory");
+  }
+  __syncwarp();
+  const bool done = mbar_wait_bounded(smem_addr(&bar), 0);
+  if (!__all_sync(kFullMask, done) && threadIdx.x == 0) atomicOr(err, PA_DEVERR_TIMEOUT);
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+pa_status pa_pool_create(int64_t num_blocks, int32_t block_size, int32_t heads, int32_t head_dim,
+                         int32_t dtype, pa_pool* out) {
+  if (!out) return fail(PA_ERR_INVALID_ARG, "pa_pool_create: out is null");
+  if (num_blocks <= 0 || block_size <= 0 || heads <= 0 || head_dim <= 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_pool_create: sizes must be positive");
+  pa_pool p{};
+  p.num_blocks = num_blocks;
+  p.block_size = block_size;
+  p.heads = heads;
+  p.head_dim = head_dim;
+  p.dtype = dtype;
+  p.elem_bytes = dtype == PA_F32 ? 4 : 2;
+  p.token_stride = head_dim;
+  p.head_stride = (int64_t)block_size * head_dim;
+  p.block_stride = (int64_t)heads * block_size * head_dim;
+  p.bytes_per_pool = num_blocks * p.block_stride * p.elem_bytes;
+  pa_status st = check_pool(&p);
+  if (st != PA_OK) return st;
+  *out = p;
+  return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const pa_pool* pool, const void* k_new, const void* v_new,
+                               const int32_t* slot_mapping, int32_t num_tokens, void* k_pool,
+                               void* v_pool, void* stream) {
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: num_tokens < 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
+    return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: null pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: buffers must be 16-byte aligned");
+  DeviceState* dev;
+  if ((st = device_state(&dev)) != PA_OK) return st;
+  const int row_chunks = pool->head_dim * pool->elem_bytes / 16;
+  reshape_and_cache_kernel<<<num_tokens, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping,
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pool->heads, row_chunks,
+      pool->num_blocks * pool->block_size, dev->err);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "reshape_and_cache launch");
+}
+
+pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
+                                    int32_t max_blocks_per_seq, int32_t max_context_len,
+                                    int32_t partition_size, size_t* bytes) {
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (!bytes) return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bytes is null");
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bad size");
+  const int ps = resolve_partition(partition_size);
+  if (ps < kBlock || ps % kBlock != 0 || ps > kMaxPartition)
+    return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
+  const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
+  const int max_parts = std::max(1, (maxL + ps - 1) / ps);
+  *bytes = layout_for(num_seqs, pool->heads, max_parts, pool->head_dim).total;
+  return PA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validate the sizes shared by the plan and run halves and fill the
+// workspace pointers of a.
+pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_blocks_per_seq,
+                         int32_t max_context_len, int32_t partition_size, void* workspace,
+                         size_t workspace_bytes, DecodeArgs* a, DeviceState** dev) {
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "decode: bad size");
+  const int ps = resolve_partition(partition_size);
+  if (ps < kBlock || ps % kBlock != 0 || ps > kMaxPartition)
+    return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
+  const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
+  const int max_parts = std::max(1, (maxL + ps - 1) / ps);
+  const WorkspaceLayout w = layout_for(num_seqs, pool->heads, max_parts, pool->head_dim);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(PA_ERR_WORKSPACE, "decode: workspace missing, not 256-byte aligned or too small");
+  if ((st = device_state(dev)) != PA_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  *a = DecodeArgs{};
+  a->plan = reinterpret_cast<PlanHeader*>(ws + w.header);
+  a->lens = reinterpret_cast<int32_t*>(ws + w.lens);
+  a->nparts = reinterpret_cast<int32_t*>(ws + w.nparts);
+  a->pairs = reinterpret_cast<int2*>(ws + w.pairs);
+  a->part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
+  a->part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+  a->err = (*dev)->err;
+  a->num_blocks = pool->num_blocks;
+  a->max_blocks_per_seq = max_blocks_per_seq;
+  a->num_seqs = num_seqs;
+  a->heads = pool->heads;
+  a->head_groups = (pool->heads + kDecodeWarps - 1) / kDecodeWarps;
+  a->partition_size = ps;
+  a->max_parts = max_parts;
+  a->max_context_len = maxL;
+  return PA_OK;
+}
+
+pa_status launch_plan(const DecodeArgs& a, cudaStream_t s) {
+  decode_plan_kernel<<<1, 1024, (a.partition_size / kBlock + 1) * sizeof(int32_t), s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode plan launch");
+}
+
+pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState& dev,
+                     cudaStream_t s) {
+  cudaError_t e;
+  switch (pool->dtype * 1000 + pool->head_dim) {
+    case PA_F32 * 1000 + 64: e = launch_decode<float, 64>(a, dev, s); break;
+    case PA_F32 * 1000 + 128: e = launch_decode<float, 128>(a, dev, s); break;
+    case PA_F16 * 1000 + 64: e = launch_decode<__half, 64>(a, dev, s); break;
+    case PA_F16 * 1000 + 128: e = launch_decode<__half, 128>(a, dev, s); break;
+    case PA_BF16 * 1000 + 64: e = launch_decode<__nv_bfloat16, 64>(a, dev, s); break;
+    case PA_BF16 * 1000 + 128: e = launch_decode<__nv_bfloat16, 128>(a, dev, s); break;
+    default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
+  }
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode launch");
+}
+
+pa_status check_run_pointers(const void* q, const void* k_pool, const void* v_pool,
+                             const int32_t* block_tables, const void* out, float scale) {
+  if (!q || !k_pool || !v_pool || !block_tables || !out)
+    return fail(PA_ERR_INVALID_ARG, "decode: null pointer");
+  if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out))
+    return fail(PA_ERR_INVALID_ARG, "decode: q, pools and out must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "decode: scale not finite");
+  return PA_OK;
+}
+
+void set_run_args(DecodeArgs* a, const void* q, const void* k_pool, const void* v_pool,
+                  const int32_t* block_tables, void* out, float scale) {
+  a->q = q;
+  a->k_pool = k_pool;
+  a->v_pool = v_pool;
+  a->block_tables = block_tables;
+  a->out = out;
+  a->scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32_t num_seqs,
+                         int32_t max_blocks_per_seq, int32_t max_context_len,
+                         int32_t partition_size, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (num_seqs == 0) return check_pool(pool);
+  if (!context_lens) return fail(PA_ERR_INVALID_ARG, "pa_decode_plan: context_lens is null");
+  DecodeArgs a;
+  DeviceState* dev;
+  pa_status st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len,
+                                partition_size, workspace, workspace_bytes, &a, &dev);
+  if (st != PA_OK) return st;
+  a.context_lens = context_lens;
+  return launch_plan(a, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const void* k_pool,
+                                      const void* v_pool, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, int32_t num_seqs,
+                                      int32_t max_context_len, float scale, void* out,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t partition_size, void* stream) {
+  if (num_seqs == 0) return check_pool(pool);
+  pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
+  if (st != PA_OK) return st;
+  DecodeArgs a;
+  DeviceState* dev;
+  st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+                      workspace, workspace_bytes, &a, &dev);
+  if (st != PA_OK) return st;
+  set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
+  return launch_run(pool, a, *dev, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_pool,
+                              const void* v_pool, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t max_context_len, float scale, void* out,
+                              void* workspace, size_t workspace_bytes, int32_t partition_size,
+                              void* stream) {
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: num_seqs < 0");
+  if (num_seqs == 0) return check_pool(pool);
+  pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
+  if (st != PA_OK) return st;
+  if (!context_lens) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: null pointer");
+  DecodeArgs a;
+  DeviceState* dev;
+  st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+                      workspace, workspace_bytes, &a, &dev);
+  if (st != PA_OK) return st;
+  a.context_lens = context_lens;
+  set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = launch_plan(a, s)) != PA_OK) return st;
+  return launch_run(pool, a, *dev, s);
+}
+
+pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,
+                         int32_t num_pairs, void* stream) {
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: num_pairs < 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!k_pool || !v_pool || !pairs) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: null pointer");
+  if (!aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: pools must be 16-byte aligned");
+  DeviceState* dev;
+  if ((st = device_state(&dev)) != PA_OK) return st;
+  const int64_t block_chunks = pool->block_stride * pool->elem_bytes / 16;
+  const int split = (int)std::min<int64_t>(16, std::max<int64_t>(1, block_chunks / 1024));
+  copy_blocks_kernel<<<dim3(num_pairs, split), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, pool->num_blocks,
+      block_chunks, dev->err);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks launch");
+}
+
+pa_status pa_selftest_wait_timeout(void* stream) {
+  DeviceState* dev;
+  pa_status st = device_state(&dev);
+  if (st != PA_OK) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->err);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "selftest launch");
+}
+
+pa_status pa_device_errors(void* stream, uint32_t* flags) {
+  if (!flags) return fail(PA_ERR_INVALID_ARG, "pa_device_errors: flags is null");
+  *flags = 0;
+  DeviceState* dev;
+  pa_status st = device_state(&dev);
+  if (st != PA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, dev->err, sizeof v, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dev->err, 0, sizeof v, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "pa_device_errors");
+  *flags = v;
+  if (v & PA_DEVERR_TIMEOUT) return fail(PA_ERR_TIMEOUT, "a device-side wait timed out");
+  if (v) return fail(PA_ERR_OUT_OF_BOUNDS, "a device-side bounds check fired");
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -25,3 +25,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Compile the CUDA library and the C oracle in-tree if they are stale."""
+    from paged_kv_cache_478_b200 import build as pa_build
+
+    import oracle
+
+    pa_build.build()
+    oracle.build()

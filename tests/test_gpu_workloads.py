@@ -1,0 +1,226 @@
+"""The three larger workloads through the C ABI against the oracle.
+
+  * shared prefix + copy-on-write: 128 sequences share a 1000-token system
+    prefix (63 blocks, the last one partial); each appends a suffix of 1 to
+    512 tokens, which copies the partial block on the first divergent write
+    ("Atención paginada en modelos de lenguaje grandes (LLM)", 7minutos.es,
+    section 3; "PagedAttention" wiki mirror, "Descripció");
+  * long context split-K: 8 sequences x 32768 tokens, partitions of 512;
+  * the full 32-layer decode step at the pages' scale (200 requests, 32 x 32
+    x 128 fp16), checked on sampled layers and sequences, in the launch
+    configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_478_b200 as pa
+from paged_kv_cache_478_b200 import synthetic as syn
+from tests.gpu_cases import assert_parity, bits, dev, host, workspace_for
+
+pytestmark = pytest.mark.gpu
+
+BS = 16
+
+
+def _gpu_shared_prefix(case, nb, private_prefix=False):
+    """Product side: C++ block manager + reshape_and_cache + copy_blocks +
+    decode.  With private_prefix every sequence gets its own copy of the
+    prefix instead of sharing it."""
+    S, H, D = case["q"].shape
+    P = case["prefix_len"]
+    bm = pa.BlockManager(nb)
+    maxb = math.ceil((P + 512) / BS)
+    tables = np.full((S, maxb), -1, dtype=np.int32)
+    kp = torch.zeros((nb, H, BS, D), dtype=torch.float16, device="cuda")
+    vp = torch.zeros_like(kp)
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    lens = np.zeros(S, dtype=np.int32)
+    kpre, vpre = dev(case["k_prefix"]), dev(case["v_prefix"])
+    if private_prefix:
+        for s in range(S):
+            lens[s], slots, _ = bm.append_tokens(tables[s], 0, P)
+            pa.pa_reshape_and_cache(pool, kpre, vpre, dev(slots), kp, vp)
+    else:
+        lens[0], slots, _ = bm.append_tokens(tables[0], 0, P)
+        for s in range(1, S):
+            bm.fork_table(tables[0], math.ceil(P / BS), tables[s])
+            lens[s] = P
+        pa.pa_reshape_and_cache(pool, kpre, vpre, dev(slots), kp, vp)
+    all_slots, all_pairs = [], []
+    for s in range(S):
+        lens[s], slots, pairs = bm.append_tokens(tables[s], int(lens[s]),
+                                                 int(case["suffix_lens"][s]))
+        all_slots.append(slots)
+        all_pairs.append(pairs)
+    pairs = np.concatenate(all_pairs).reshape(-1, 2).astype(np.int32)
+    if len(pairs):
+        pa.pa_copy_blocks(pool, kp, vp, dev(pairs))
+    pa.pa_reshape_and_cache(pool, dev(np.concatenate(case["k_suffix"])),
+                            dev(np.concatenate(case["v_suffix"])),
+                            dev(np.concatenate(all_slots)), kp, vp)
+    q = dev(case["q"])
+    out = torch.empty_like(q)
+    ws = workspace_for(pool, S, maxb)
+    pa.pa_decode_attention(pool, q, kp, vp, dev(tables), dev(lens), case["scale"], out, ws)
+    assert pa.pa_device_errors() == 0
+    return dict(out=out, kp=kp, vp=vp, tables=tables, lens=lens, pairs=pairs, bm=bm, pool=pool,
+                ws=ws, slots=all_slots)
+
+
+def _oracle_shared_prefix(case, nb):
+    """Oracle side: page-pool model + host scatter/copy + fp64 attention."""
+    S, H, D = case["q"].shape
+    P = case["prefix_len"]
+    pp = oracle.PagePool(nb)
+    reqs = [oracle.PagedRequest(pp) for _ in range(S)]
+    kp = np.zeros((nb, H, BS, D), dtype=np.float16)
+    vp = np.zeros_like(kp)
+    slots = np.array([reqs[0].generate_token()[0] for _ in range(P)], dtype=np.int32)
+    for s in range(1, S):
+        reqs[s].share_prefix_of(reqs[0])
+    oracle.reshape_and_cache(case["k_prefix"], case["v_prefix"], slots, kp, vp)
+    all_slots, pairs = [], []
+    for s in range(S):
+        for _ in range(int(case["suffix_lens"][s])):
+            slot, cow = reqs[s].generate_token()
+            all_slots.append(slot)
+            if cow is not None:
+                pairs.append(cow)
+    pairs = np.array(pairs, dtype=np.int32).reshape(-1, 2)
+    oracle.copy_blocks(kp, vp, pairs)
+    oracle.reshape_and_cache(np.concatenate(case["k_suffix"]), np.concatenate(case["v_suffix"]),
+                             np.array(all_slots, dtype=np.int32), kp, vp)
+    maxb = math.ceil((P + 512) / BS)
+    tables = np.full((S, maxb), -1, dtype=np.int32)
+    for s, r in enumerate(reqs):
+        tables[s, :len(r.block_table)] = r.block_table
+    lens = np.array([r.num_tokens for r in reqs], dtype=np.int32)
+    out = oracle.decode_attention(case["q"], kp, vp, tables, lens, case["scale"])
+    return dict(out=out, kp=kp, vp=vp, tables=tables, lens=lens, pairs=pairs)
+
+
+def test_shared_prefix_copy_on_write():
+    case = syn.shared_prefix_case(seed=0)
+    S = 128
+    nb = 63 + S + sum(math.ceil(int(n) / BS) for n in case["suffix_lens"])
+    g = _gpu_shared_prefix(case, nb)
+    r = _oracle_shared_prefix(case, nb)
+    # block management: identical tables, lengths and copy pairs
+    assert np.array_equal(g["tables"], r["tables"])
+    assert np.array_equal(g["lens"], r["lens"])
+    assert np.array_equal(g["pairs"], r["pairs"])
+    assert len(g["pairs"]) == S - 1  # the last holder writes block 62 in place
+    assert all(p[0] == 62 for p in g["pairs"])
+    # device state after copy_blocks + reshape_and_cache: bit-exact
+    assert np.array_equal(bits(g["kp"]), bits(r["kp"]))
+    assert np.array_equal(bits(g["vp"]), bits(r["vp"]))
+    assert_parity(g["out"], r["out"], "shared prefix")
+
+    # shared prefix == private copies of the prefix, bit for bit
+    nb2 = S * 64 + S + sum(math.ceil(int(n) / BS) for n in case["suffix_lens"])
+    priv = _gpu_shared_prefix(case, nb2, private_prefix=True)
+    assert torch.equal(priv["out"], g["out"])
+
+    # copy-on-write leaves every other sequence's output unchanged: fork
+    # sequence 10 (its blocks become shared) and let the fork write one token
+    bm, pool, tables, lens = g["bm"], g["pool"], g["tables"], g["lens"]
+    fork = np.full(tables.shape[1], -1, dtype=np.int32)
+    n10 = math.ceil(int(lens[10]) / BS)
+    bm.fork_table(tables[10], n10, fork)
+    L_fork, slots, pairs = bm.append_tokens(fork, int(lens[10]), 1)
+    if int(lens[10]) % BS:
+        assert len(pairs) == 1 and bm.refcount(int(tables[10][n10 - 1])) == 1
+        pa.pa_copy_blocks(pool, g["kp"], g["vp"], dev(pairs))
+    rng = np.random.default_rng(1)
+    kn = rng.standard_normal((1, 32, 128)).astype(np.float16)
+    pa.pa_reshape_and_cache(pool, dev(kn), dev(kn), dev(slots), g["kp"], g["vp"])
+    tables2 = np.vstack([tables, fork[None]])
+    lens2 = np.append(lens, L_fork).astype(np.int32)
+    q2 = torch.cat([dev(case["q"]), dev(case["q"][10:11])])
+    out2 = torch.empty_like(q2)
+    ws2 = workspace_for(pool, S + 1, tables.shape[1])
+    pa.pa_decode_attention(pool, q2, g["kp"], g["vp"], dev(tables2), dev(lens2), case["scale"],
+                           out2, ws2)
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(out2[:S], g["out"])
+
+
+def test_long_context_split_k():
+    S, H, D, CTX = 8, 32, 128, 32768
+    lens, tables, nb = syn.long_context_tables(seed=0, num_seqs=S, context=CTX)
+    kp = torch.empty((nb, H, BS, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 101)
+    syn.fill_normal_device(vp, 102)
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((S, H, D)).astype(np.float16)
+    kn = rng.standard_normal((S, H, D)).astype(np.float16)
+    vn = rng.standard_normal((S, H, D)).astype(np.float16)
+    sample = [0, 5]
+    kh, vh = host(kp), host(vp)  # oracle inputs: the pools as drawn, before any kernel
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    slots = pa.pa_decode_slots(tables, lens)
+    pa.pa_reshape_and_cache(pool, dev(kn), dev(vn), dev(slots), kp, vp)
+    out = torch.empty((S, H, D), dtype=torch.float16, device="cuda")
+    ws = workspace_for(pool, S, tables.shape[1], 0, 512)
+    pa.pa_decode_attention(pool, dev(q), kp, vp, dev(tables), dev(lens), 1 / math.sqrt(D), out, ws,
+                           partition_size=512)
+    assert pa.pa_device_errors() == 0
+    oslots = np.array([oracle.slot_of_c(tables[s], CTX - 1) for s in range(S)], dtype=np.int32)
+    oracle.reshape_and_cache(kn, vn, oslots, kh, vh)
+    only = np.zeros(S, dtype=np.int32)
+    only[sample] = lens[sample]
+    ref = oracle.decode_attention(q, kh, vh, tables, only, 1 / math.sqrt(D))
+    assert_parity(out[sample], ref[sample], "long context")
+    # the new tokens landed where the oracle put them
+    for s in range(S):
+        b, o = divmod(int(oslots[s]), BS)
+        assert np.array_equal(bits(kp[b, :, o]), bits(kn[s]))
+
+
+def test_full_decode_step_sampled():
+    """200 requests x 32 layers x 32 heads x 128 fp16, one block-id space for
+    every layer; per layer reshape_and_cache of the new token then decode,
+    launched exactly as the benchmark launches them.  Layers 0 and 31 and
+    eight sequences are checked against the oracle."""
+    S, H, D, LAYERS = 200, 32, 128, 32
+    lens = syn.full_step_lengths(seed=0, num_seqs=S)
+    tables, nb = syn.full_step_tables(0, lens)
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    slots = dev(pa.pa_decode_slots(tables, lens))
+    btd, cld = dev(tables), dev(lens)
+    ws = workspace_for(pool, S, tables.shape[1])
+    rng = np.random.default_rng(0)
+    sample_layers = [0, LAYERS - 1]
+    sample_seqs = sorted(rng.choice(S, 8, replace=False).tolist())
+    checked = 0
+    for layer in range(LAYERS):
+        kp = torch.empty((nb, H, BS, D), dtype=torch.float16, device="cuda")
+        vp = torch.empty_like(kp)
+        syn.fill_normal_device(kp, 1000 + 2 * layer)
+        syn.fill_normal_device(vp, 1001 + 2 * layer)
+        q = torch.empty((S, H, D), dtype=torch.float16, device="cuda")
+        kn, vn = torch.empty_like(q), torch.empty_like(q)
+        for t, sd in ((q, 3000), (kn, 4000), (vn, 5000)):
+            syn.fill_normal_device(t, sd + layer)
+        if layer in sample_layers:
+            kh, vh = host(kp), host(vp)
+        out = torch.empty_like(q)
+        pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp)
+        pa.pa_decode_attention(pool, q, kp, vp, btd, cld, 1 / math.sqrt(D), out, ws)
+        assert pa.pa_device_errors() == 0
+        if layer in sample_layers:
+            oslots = np.array([oracle.slot_of_c(tables[s], int(lens[s]) - 1) for s in range(S)],
+                              dtype=np.int32)
+            oracle.reshape_and_cache(host(kn), host(vn), oslots, kh, vh)
+            only = np.zeros(S, dtype=np.int32)
+            only[sample_seqs] = lens[sample_seqs]
+            ref = oracle.decode_attention(host(q), kh, vh, tables, only, 1 / math.sqrt(D))
+            assert_parity(out[sample_seqs], ref[sample_seqs], f"layer {layer}")
+            checked += 1
+        del kp, vp
+    assert checked == len(sample_layers)
