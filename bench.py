@@ -46,7 +46,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_kernel_full_step.md"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partition-size", type=int, default=0)
@@ -279,7 +279,7 @@ def run_ours(args):
     uuid = torch.cuda.get_device_properties(dev).uuid
     sampler = ClockSampler(f"GPU-{uuid}" if not str(uuid).startswith("GPU-") else str(uuid))
     sampler.start()
-    time.sleep(0.5)
+    time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
