@@ -165,6 +165,31 @@ pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const 
                                       int32_t partition_size, void* stream);
 
 /*
+ * Decode attention that allocates nothing.  Same computation, arguments and
+ * errors as pa_decode_attention, minus the workspace: the plan and split-K
+ * partials live in a static device buffer inside the library of
+ * PA_STATIC_SCRATCH_BYTES (32 MiB), which every GPU that loads the library
+ * holds until the process exits.  No counterpart on the pages: it exists for
+ * callers that may not call cudaMalloc, such as plugins hosted by a runtime
+ * that owns all device memory through its own pool, or latency-bound loops
+ * that cannot afford cudaMalloc's implicit device synchronisation.
+ * Sizes whose workspace (pa_decode_workspace_bytes) exceeds the buffer are
+ * rejected with PA_ERR_WORKSPACE before anything is launched.
+ * The first call on each device resolves the buffer's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one buffer: calls that overlap on the GPU (different
+ * streams, or different threads without ordering) race and corrupt each
+ * other's results; order them on one stream.  The buffer keeps the last
+ * call's contents; each call rewrites every part it reads.
+ */
+#define PA_STATIC_SCRATCH_BYTES (32u << 20)
+pa_status pa_decode_attention_static(const pa_pool* pool, const void* q, const void* k_pool,
+                                     const void* v_pool, const int32_t* block_tables,
+                                     int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                     int32_t num_seqs, int32_t max_context_len, float scale,
+                                     void* out, int32_t partition_size, void* stream);
+
+/*
  * Block-granular copy-on-write, device half ("PagedAttention" wiki mirror,
  * "Descripció"; 7minutos.es section 3, cow_copy): for each (src, dst) row of
  * pairs (device int32 [num_pairs][2]) copy the whole physical block, every

@@ -75,6 +75,8 @@ def lib():
             "pa_decode_plan": [P(pa_pool), vp, i32, i32, i32, i32, vp, sz, vp],
             "pa_decode_attention_planned": [P(pa_pool), vp, vp, vp, vp, i32, i32, i32,
                                             ctypes.c_float, vp, vp, sz, i32, vp],
+            "pa_decode_attention_static": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, i32,
+                                           ctypes.c_float, vp, i32, vp],
             "pa_copy_blocks": [P(pa_pool), vp, vp, vp, i32, vp],
             "pa_device_errors": [vp, P(ctypes.c_uint32)],
             "pa_selftest_wait_timeout": [vp],
@@ -233,6 +235,30 @@ def pa_decode_attention_planned(pool, q, k_pool, v_pool, block_tables, scale, ou
         _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], S,
         max_context_len, float(scale), _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def pa_decode_attention_static(pool, q, k_pool, v_pool, block_tables, context_lens, scale, out,
+                               max_context_len=0, partition_size=0, stream=None):
+    """pa_decode_attention without a workspace: the library's static scratch
+    buffer (STATIC_SCRATCH_BYTES per GPU) holds the plan and the partials, so
+    neither the caller nor the library allocates.  Calls must not overlap on
+    the GPU; the first call on a device must come before any stream capture."""
+    torch = _torch()
+    S = q.shape[0]
+    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
+    dt = _pool_torch_dtype(pool)
+    _check(lib().pa_decode_attention_static(
+        ctypes.byref(pool), _dev_ptr(q, "q", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
+        _check_pool_tensor(pool, v_pool, "v_pool"),
+        _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev_ptr(context_lens, "context_lens", torch.int32), S, max_context_len, float(scale),
+        _dev_ptr(out, "out", dt), partition_size, _stream(stream)))
 
 
 def pa_copy_blocks(pool, k_pool, v_pool, pairs, stream=None):

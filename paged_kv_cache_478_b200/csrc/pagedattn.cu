@@ -405,6 +405,70 @@ pa_status pa_selftest_wait_timeout(void* stream) {
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "selftest launch");
 }
 
+}  // extern "C"
+
+// ---- decode with a static scratch buffer (no allocation by anyone) ----------------------
+// For callers that may not call cudaMalloc: plugins whose host runtime owns
+// all device memory, and loops that cannot pay cudaMalloc's implicit device
+// synchronisation.  The plan and the split-K partials live in this buffer.
+// Every call shares it, so calls that overlap on the GPU race; the plan
+// kernel rewrites the header and counters it needs at the start of each call.
+static __device__ __align__(256) uint8_t g_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_static_scratch, resolved once per device with that
+// device current (the host-side symbol is only a stand-in, never a device
+// address).
+void* g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_mutex;
+
+pa_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "device index out of range");
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_static_scratch)");
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_attention_static(const pa_pool* pool, const void* q, const void* k_pool,
+                                     const void* v_pool, const int32_t* block_tables,
+                                     int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                     int32_t num_seqs, int32_t max_context_len, float scale,
+                                     void* out, int32_t partition_size, void* stream) {
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: num_seqs < 0");
+  size_t need = 0;
+  pa_status st = pa_decode_workspace_bytes(pool, num_seqs, max_blocks_per_seq, max_context_len,
+                                           partition_size, &need);
+  if (st != PA_OK) return st;
+  if (need > PA_STATIC_SCRATCH_BYTES) {
+    char buf[256];
+    std::snprintf(buf, sizeof buf,
+                  "pa_decode_attention_static: these sizes need %zu bytes of scratch; the static "
+                  "buffer holds %u (use fewer sequences or a larger partition_size, or "
+                  "pa_decode_attention with a caller workspace)",
+                  need, PA_STATIC_SCRATCH_BYTES);
+    return fail(PA_ERR_WORKSPACE, buf);
+  }
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != PA_OK) return st;
+  return pa_decode_attention(pool, q, k_pool, v_pool, block_tables, max_blocks_per_seq,
+                             context_lens, num_seqs, max_context_len, scale, out, scratch,
+                             PA_STATIC_SCRATCH_BYTES, partition_size, stream);
+}
+
 pa_status pa_device_errors(void* stream, uint32_t* flags) {
   if (!flags) return fail(PA_ERR_INVALID_ARG, "pa_device_errors: flags is null");
   *flags = 0;
