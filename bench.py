@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="layers per step (profiling a smaller case; the bench line uses 32)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -233,15 +235,16 @@ def run_ours(args):
     lens = syn.full_step_lengths(seed=rank, num_seqs=S)
     tables, nb = syn.full_step_tables(rank, lens)
     pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    n_layers = args.layers
     kpools, vpools = [], []
-    for layer in range(LAYERS):
+    for layer in range(n_layers):
         kp = torch.empty((nb, H, BS, D), dtype=torch.float16, device=dev)
         vp = torch.empty_like(kp)
         syn.fill_normal_device(kp, 1000 * (rank + 1) + 2 * layer)
         syn.fill_normal_device(vp, 1000 * (rank + 1) + 2 * layer + 1)
         kpools.append(kp)
         vpools.append(vp)
-    q = torch.empty((LAYERS, S, H, D), dtype=torch.float16, device=dev)
+    q = torch.empty((n_layers, S, H, D), dtype=torch.float16, device=dev)
     k_new, v_new = torch.empty_like(q), torch.empty_like(q)
     for t, sd in ((q, 7), (k_new, 8), (v_new, 9)):
         syn.fill_normal_device(t, 100 * (rank + 1) + sd)
@@ -254,13 +257,13 @@ def run_ours(args):
                      dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(D)
     max_parts = math.ceil(tables.shape[1] * BS / (ps or 256))
-    kernels_per_step = 1 + LAYERS * (2 + (1 if max_parts > 1 else 0))
+    kernels_per_step = 1 + n_layers * (2 + (1 if max_parts > 1 else 0))
 
     ev_pairs = []
 
     def step(record=False):
         pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=ps)
-        for layer in range(LAYERS):
+        for layer in range(n_layers):
             pa.pa_reshape_and_cache(pool, k_new[layer], v_new[layer], slots, kpools[layer],
                                     vpools[layer])
             if record:
@@ -303,7 +306,7 @@ def run_ours(args):
     decode_avg_ms = float(np.mean(decode_ms))
 
     ms_per_step = elapsed_ms / args.steps
-    step_kv = kv_bytes(lens) * LAYERS
+    step_kv = kv_bytes(lens) * n_layers
     value = step_kv * world / (ms_per_step * 1e-3) / 1e9
     tokens_per_s = S * world / (ms_per_step * 1e-3)
     peaks, peak_kind = measured_peaks()
@@ -328,7 +331,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "num_seqs": S, "layers": LAYERS, "heads": H,
+            "config": {"workload": WORKLOAD, "num_seqs": S, "layers": n_layers, "heads": H,
                        "head_dim": D, "block_size": BS, "cached_tokens": int(lens.sum()),
                        "pool_blocks": nb, "partition_size": ps or 256,
                        "kv_bytes_per_step": step_kv, "l2": "inputs larger than L2 (no flush)",
@@ -361,17 +364,18 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
     so layer l+1's inputs cross PCIe while layer l computes."""
     import torch.distributed as dist
 
+    n_layers = len(kpools)
     main = torch.cuda.current_stream()
     copy = torch.cuda.Stream(device=dev)
     rng = np.random.default_rng(11)
-    h_q = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
-    h_k = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
-    h_v = torch.from_numpy(rng.standard_normal((LAYERS, S, H, D)).astype(np.float16)).pin_memory()
-    h_out = torch.empty((LAYERS, S, H, D), dtype=torch.float16).pin_memory()
+    h_q = torch.from_numpy(rng.standard_normal((n_layers, S, H, D)).astype(np.float16)).pin_memory()
+    h_k = torch.from_numpy(rng.standard_normal((n_layers, S, H, D)).astype(np.float16)).pin_memory()
+    h_v = torch.from_numpy(rng.standard_normal((n_layers, S, H, D)).astype(np.float16)).pin_memory()
+    h_out = torch.empty((n_layers, S, H, D), dtype=torch.float16).pin_memory()
     h_bt = torch.from_numpy(tables).pin_memory()
     h_cl = torch.from_numpy(lens).pin_memory()
     h_slots = torch.empty(S, dtype=torch.int32).pin_memory()
-    d_q = torch.empty((LAYERS, S, H, D), dtype=torch.float16, device=dev)
+    d_q = torch.empty((n_layers, S, H, D), dtype=torch.float16, device=dev)
     d_k, d_v, d_out = torch.empty_like(d_q), torch.empty_like(d_q), torch.empty_like(d_q)
     d_bt = torch.empty_like(h_bt, device=dev)
     d_cl = torch.empty_like(h_cl, device=dev)
@@ -387,7 +391,7 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
             d_bt.copy_(h_bt, non_blocking=True)
             d_cl.copy_(h_cl, non_blocking=True)
             d_slots.copy_(h_slots, non_blocking=True)
-            for layer in range(LAYERS):
+            for layer in range(n_layers):
                 d_q[layer].copy_(h_q[layer], non_blocking=True)
                 d_k[layer].copy_(h_k[layer], non_blocking=True)
                 d_v[layer].copy_(h_v[layer], non_blocking=True)
@@ -396,7 +400,7 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
                 in_ready.append(ev)
         main.wait_event(in_ready[0])
         pa.pa_decode_plan(pool, d_cl, tables.shape[1], ws, partition_size=ps)
-        for layer in range(LAYERS):
+        for layer in range(n_layers):
             main.wait_event(in_ready[layer])
             pa.pa_reshape_and_cache(pool, d_k[layer], d_v[layer], d_slots, kpools[layer],
                                     vpools[layer])
@@ -426,7 +430,7 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     assert torch.isfinite(h_out.float()).all()
-    value = kv_bytes(lens) * LAYERS * world / (ms * 1e-3) / 1e9
+    value = kv_bytes(lens) * n_layers * world / (ms * 1e-3) / 1e9
     return {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
             "decode_tokens_per_s": round(S * world / (ms * 1e-3), 1)}
