@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers per step (profiling a smaller case; the bench line uses 32)")
+    ap.add_argument("--path", choices=["fused", "separate"], default="fused",
+                    help="fused: one append+attend launch per layer; separate: "
+                         "reshape_and_cache then decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -213,6 +216,35 @@ def run_reference(args):
 
 # ---- our CUDA path -------------------------------------------------------------------------
 
+def replica_workload(rank):
+    """The requests rank `rank` owns: its own 200 sequences (seed = rank),
+    lengths, block tables and pool size.  Replicas share nothing."""
+    from paged_kv_cache_478_b200 import synthetic as syn
+
+    lens = syn.full_step_lengths(seed=rank, num_seqs=S)
+    tables, nb = syn.full_step_tables(rank, lens)
+    return lens, tables, nb
+
+
+def max_over_ranks(value, device=None):
+    """Max of a per-rank time over all ranks (the only collective)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(step_kv_bytes_per_rank, world, ms_per_step):
+    """Whole-job KV GB/s and tokens/s: every rank processed its own step in
+    at most ms_per_step (the max over ranks)."""
+    sec = ms_per_step * 1e-3
+    return step_kv_bytes_per_rank * world / sec / 1e9, S * world / sec
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -232,8 +264,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     # every rank owns its own 200 requests (weak scaling): seed = rank
-    lens = syn.full_step_lengths(seed=rank, num_seqs=S)
-    tables, nb = syn.full_step_tables(rank, lens)
+    lens, tables, nb = replica_workload(rank)
     pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
     n_layers = args.layers
     kpools, vpools = [], []
@@ -256,21 +287,28 @@ def run_ours(args):
     ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, ps),
                      dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(D)
-    max_parts = math.ceil(tables.shape[1] * BS / (ps or 256))
-    kernels_per_step = 1 + n_layers * (2 + (1 if max_parts > 1 else 0))
+    kernels_per_step = 1 + n_layers * (1 if args.path == "fused" else 2)
 
     ev_pairs = []
+
+    fused = args.path == "fused"
 
     def step(record=False):
         pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=ps)
         for layer in range(n_layers):
-            pa.pa_reshape_and_cache(pool, k_new[layer], v_new[layer], slots, kpools[layer],
-                                    vpools[layer])
+            if not fused:
+                pa.pa_reshape_and_cache(pool, k_new[layer], v_new[layer], slots, kpools[layer],
+                                        vpools[layer])
             if record:
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            pa.pa_decode_attention_planned(pool, q[layer], kpools[layer], vpools[layer], bt, scale,
-                                           out[layer], ws, partition_size=ps)
+            if fused:  # reshape_and_cache of the new token + decode in one launch
+                pa.pa_decode_append_attention_planned(pool, q[layer], k_new[layer], v_new[layer],
+                                                      kpools[layer], vpools[layer], bt, scale,
+                                                      out[layer], ws, partition_size=ps)
+            else:
+                pa.pa_decode_attention_planned(pool, q[layer], kpools[layer], vpools[layer], bt,
+                                               scale, out[layer], ws, partition_size=ps)
             if record:
                 e1.record(stream)
                 ev_pairs.append((e0, e1))
@@ -295,11 +333,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     errs = pa.pa_device_errors()
     assert errs == 0, f"device error bits {errs:#x}"
     decode_ms = [a.elapsed_time(b) for a, b in ev_pairs]
@@ -307,8 +341,7 @@ def run_ours(args):
 
     ms_per_step = elapsed_ms / args.steps
     step_kv = kv_bytes(lens) * n_layers
-    value = step_kv * world / (ms_per_step * 1e-3) / 1e9
-    tokens_per_s = S * world / (ms_per_step * 1e-3)
+    value, tokens_per_s = job_throughput(step_kv, world, ms_per_step)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     per_launch = algorithmic_bytes_per_launch(lens)
@@ -333,9 +366,9 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "num_seqs": S, "layers": n_layers, "heads": H,
                        "head_dim": D, "block_size": BS, "cached_tokens": int(lens.sum()),
-                       "pool_blocks": nb, "partition_size": ps or 256,
+                       "pool_blocks": nb, "partition_size": ps or "auto",
                        "kv_bytes_per_step": step_kv, "l2": "inputs larger than L2 (no flush)",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}", "path": args.path},
             "decode_tokens_per_s": round(tokens_per_s, 1),
             "pct_of_hbm_peak": round(100 * value / world / peak, 2),
             "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
@@ -343,7 +376,8 @@ def run_ours(args):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": committed_traffic(),
                          "peak_kind": peak_kind,
-                         "kernel": "paged_decode_kernel + merge (events bracket one planned call)",
+                         "kernel": "paged_decode_kernel (events bracket one planned call: "
+                                   + ("append + attend" if fused else "attend") + ")",
                          "bytes_per_launch": per_launch,
                          "avg_launch_ms": round(decode_avg_ms, 5)},
             "gpu_launches": kernels_per_step * args.steps,
@@ -381,16 +415,19 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
     d_cl = torch.empty_like(h_cl, device=dev)
     d_slots = torch.empty(S, dtype=torch.int32, device=dev)
     scale = 1.0 / math.sqrt(D)
-    h2d = 3 * d_q.numel() * 2 + h_bt.numel() * 4 + h_cl.numel() * 4 + S * 4
+    fused = args.path == "fused"
+    h2d = 3 * d_q.numel() * 2 + h_bt.numel() * 4 + h_cl.numel() * 4 + (0 if fused else S * 4)
     d2h = d_out.numel() * 2
 
     def step():
-        h_slots.copy_(torch.from_numpy(pa.pa_decode_slots(tables, lens)))  # host scheduler work
+        if not fused:  # the fused kernel finds each new token's slot itself
+            h_slots.copy_(torch.from_numpy(pa.pa_decode_slots(tables, lens)))
         in_ready = []
         with torch.cuda.stream(copy):
             d_bt.copy_(h_bt, non_blocking=True)
             d_cl.copy_(h_cl, non_blocking=True)
-            d_slots.copy_(h_slots, non_blocking=True)
+            if not fused:
+                d_slots.copy_(h_slots, non_blocking=True)
             for layer in range(n_layers):
                 d_q[layer].copy_(h_q[layer], non_blocking=True)
                 d_k[layer].copy_(h_k[layer], non_blocking=True)
@@ -402,10 +439,15 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
         pa.pa_decode_plan(pool, d_cl, tables.shape[1], ws, partition_size=ps)
         for layer in range(n_layers):
             main.wait_event(in_ready[layer])
-            pa.pa_reshape_and_cache(pool, d_k[layer], d_v[layer], d_slots, kpools[layer],
-                                    vpools[layer])
-            pa.pa_decode_attention_planned(pool, d_q[layer], kpools[layer], vpools[layer], d_bt,
-                                           scale, d_out[layer], ws, partition_size=ps)
+            if args.path == "fused":
+                pa.pa_decode_append_attention_planned(pool, d_q[layer], d_k[layer], d_v[layer],
+                                                      kpools[layer], vpools[layer], d_bt, scale,
+                                                      d_out[layer], ws, partition_size=ps)
+            else:
+                pa.pa_reshape_and_cache(pool, d_k[layer], d_v[layer], d_slots, kpools[layer],
+                                        vpools[layer])
+                pa.pa_decode_attention_planned(pool, d_q[layer], kpools[layer], vpools[layer],
+                                               d_bt, scale, d_out[layer], ws, partition_size=ps)
             done = torch.cuda.Event()
             done.record(main)
             copy.wait_event(done)
@@ -424,11 +466,7 @@ def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, 
         step()
     t1.record(main)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
     assert torch.isfinite(h_out.float()).all()
     value = kv_bytes(lens) * n_layers * world / (ms * 1e-3) / 1e9
     return {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),

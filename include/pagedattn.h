@@ -106,8 +106,9 @@ pa_status pa_reshape_and_cache(const pa_pool* pool, const void* k_new, const voi
 
 /*
  * Bytes of device workspace pa_decode_attention needs for these sizes
- * (work plan + split-K partial results).  partition_size 0 = the default.
- * max_context_len 0 = max_blocks_per_seq * block_size.
+ * (work plan + split-K partial results).  With partition_size 0 the result
+ * covers every automatic choice.  max_context_len 0 = max_blocks_per_seq *
+ * block_size.
  */
 pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
                                     int32_t max_blocks_per_seq, int32_t max_context_len,
@@ -121,8 +122,11 @@ pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
  * softmax; the result is rounded to the pool dtype.  A sequence of length 0
  * gets zeros.
  * Long contexts are split into partitions of partition_size tokens (a
- * multiple of 16; 0 = default 256) whose partial results are merged by
- * log-sum-exp in a second kernel.  The work order is planned on the device
+ * multiple of 16 up to 4096) whose partial results are merged by
+ * log-sum-exp, in partition order, by the last CTA to finish a sequence.
+ * partition_size 0 chooses automatically: 512-token partitions while
+ * sequences x head groups already give two work items per resident CTA,
+ * otherwise about four items per resident CTA (never below 256 tokens).  The work order is planned on the device
  * from context_lens (longest partitions first).
  * max_context_len bounds every context_lens[s] (0 = max_blocks_per_seq *
  * block_size); a length above it or above the table width sets
@@ -163,6 +167,34 @@ pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const 
                                       int32_t max_context_len, float scale, void* out,
                                       void* workspace, size_t workspace_bytes,
                                       int32_t partition_size, void* stream);
+
+/*
+ * Fused append + attend: pa_reshape_and_cache of each sequence's new token
+ * followed by pa_decode_attention, in one pass.  k_new, v_new are
+ * [num_seqs][heads][head_dim] (pool dtype, 16-byte aligned): the token of
+ * sequence s is written at its position context_lens[s] - 1, i.e. slot
+ * block_tables[s][(L-1)/bs] * bs + (L-1) % bs, and attended to with the rest.
+ * The pools after the call, and the output, are bit-identical to the two
+ * separate calls.  Sequences of length 0 append nothing.  The block holding
+ * the new token must be private to its sequence (copy it on write first, as
+ * for pa_reshape_and_cache).  The planned form takes a plan written by
+ * pa_decode_plan, with the same rules as pa_decode_attention_planned.
+ */
+pa_status pa_decode_append_attention(const pa_pool* pool, const void* q, const void* k_new,
+                                     const void* v_new, void* k_pool, void* v_pool,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t max_context_len, float scale, void* out,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t partition_size, void* stream);
+
+pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
+                                             const void* k_new, const void* v_new, void* k_pool,
+                                             void* v_pool, const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq, int32_t num_seqs,
+                                             int32_t max_context_len, float scale, void* out,
+                                             void* workspace, size_t workspace_bytes,
+                                             int32_t partition_size, void* stream);
 
 /*
  * Decode attention that allocates nothing.  Same computation, arguments and

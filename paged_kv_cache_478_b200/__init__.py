@@ -75,6 +75,10 @@ def lib():
             "pa_decode_plan": [P(pa_pool), vp, i32, i32, i32, i32, vp, sz, vp],
             "pa_decode_attention_planned": [P(pa_pool), vp, vp, vp, vp, i32, i32, i32,
                                             ctypes.c_float, vp, vp, sz, i32, vp],
+            "pa_decode_append_attention": [P(pa_pool), vp, vp, vp, vp, vp, vp, i32, vp, i32, i32,
+                                           ctypes.c_float, vp, vp, sz, i32, vp],
+            "pa_decode_append_attention_planned": [P(pa_pool), vp, vp, vp, vp, vp, vp, i32, i32,
+                                                   i32, ctypes.c_float, vp, vp, sz, i32, vp],
             "pa_decode_attention_static": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, i32,
                                            ctypes.c_float, vp, i32, vp],
             "pa_copy_blocks": [P(pa_pool), vp, vp, vp, i32, vp],
@@ -231,6 +235,51 @@ def pa_decode_attention_planned(pool, q, k_pool, v_pool, block_tables, scale, ou
     dt = _pool_torch_dtype(pool)
     _check(lib().pa_decode_attention_planned(
         ctypes.byref(pool), _dev_ptr(q, "q", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
+        _check_pool_tensor(pool, v_pool, "v_pool"),
+        _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], S,
+        max_context_len, float(scale), _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
+
+
+def pa_decode_append_attention(pool, q, k_new, v_new, k_pool, v_pool, block_tables, context_lens,
+                               scale, out, workspace, max_context_len=0, partition_size=0,
+                               stream=None):
+    """reshape_and_cache of each sequence's new token (at position L-1) and
+    decode attention in one launch; k_new/v_new are [num_seqs, heads, head_dim]."""
+    torch = _torch()
+    S = q.shape[0]
+    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if tuple(k_new.shape) != tuple(q.shape) or tuple(v_new.shape) != tuple(q.shape):
+        raise ValueError("k_new and v_new must be [num_seqs, heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
+    dt = _pool_torch_dtype(pool)
+    _check(lib().pa_decode_append_attention(
+        ctypes.byref(pool), _dev_ptr(q, "q", dt), _dev_ptr(k_new, "k_new", dt),
+        _dev_ptr(v_new, "v_new", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
+        _check_pool_tensor(pool, v_pool, "v_pool"),
+        _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev_ptr(context_lens, "context_lens", torch.int32), S, max_context_len, float(scale),
+        _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
+
+
+def pa_decode_append_attention_planned(pool, q, k_new, v_new, k_pool, v_pool, block_tables, scale,
+                                       out, workspace, max_context_len=0, partition_size=0,
+                                       stream=None):
+    torch = _torch()
+    S = q.shape[0]
+    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if tuple(k_new.shape) != tuple(q.shape) or tuple(v_new.shape) != tuple(q.shape):
+        raise ValueError("k_new and v_new must be [num_seqs, heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S:
+        raise ValueError("block_tables must be [num_seqs, max_blocks]")
+    dt = _pool_torch_dtype(pool)
+    _check(lib().pa_decode_append_attention_planned(
+        ctypes.byref(pool), _dev_ptr(q, "q", dt), _dev_ptr(k_new, "k_new", dt),
+        _dev_ptr(v_new, "v_new", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
         _check_pool_tensor(pool, v_pool, "v_pool"),
         _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], S,
         max_context_len, float(scale), _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),

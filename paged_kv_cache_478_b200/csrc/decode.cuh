@@ -27,9 +27,15 @@
 //     ragged last partitions by decreasing size, so the tail of the grid is
 //     made of the smallest items.
 //   * Sequences with more than one partition write (m, l, unnormalised acc)
-//     per partition; the merge kernel combines them by log-sum-exp in
-//     partition order.  No atomics touch values, so results are bit-stable
-//     run to run and independent of where the blocks sit in the pool.
+//     per partition and bump a per-(sequence, head group) arrival counter;
+//     the CTA that arrives last merges all partitions by log-sum-exp in
+//     partition order and re-arms the counter (no second kernel).  No
+//     atomics touch values, so results are bit-stable run to run and
+//     independent of where the blocks sit in the pool.
+//   * Optional fused append: with k_new/v_new given, the CTA that owns a
+//     sequence's last block writes the new token's K/V row into the pool
+//     (what reshape_and_cache would do) and patches the same row of its
+//     shared-memory copy of the tile, so one launch appends and attends.
 #pragma once
 
 #include <math.h>
@@ -62,6 +68,9 @@ struct DecodeArgs {
   int2* pairs;      // [S * max_parts] work pairs (s, p)
   float2* part_ml;  // [S][H][max_parts] (running max in log2 units, sum of weights)
   float* part_acc;  // [S][H][max_parts][D] unnormalised partial outputs
+  int32_t* merge_cnt;  // [S][head_groups] partitions finished (re-armed to 0 by the merger)
+  const void* k_new;   // [S][H][D] token appended at position L-1, or null (no append)
+  const void* v_new;
   uint32_t* err;
   int64_t num_blocks;
   int32_t max_blocks_per_seq;
@@ -92,6 +101,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
       L = L < 0 ? 0 : cap;
     }
     a.lens[s] = L;
+    for (int g = 0; g < a.head_groups; ++g) a.merge_cnt[(int64_t)s * a.head_groups + g] = 0;
     const int full = L / PS, rem = L % PS;
     a.nparts[s] = max(1, full + (rem > 0 ? 1 : 0));
     if (full > 0) {
@@ -156,31 +166,73 @@ struct DecodeConfig {
   static constexpr int THREADS = WARPS * 32;
   static_assert(CPR >= 2 && CPR <= 32 && 32 % CPR == 0, "head_dim / dtype not supported");
   static_assert(NCH * 2 == CPR, "lane mapping");
+  // stage rings + one mbarrier per stage + the item's block-table slice
   static size_t smem_bytes(int partition_size) {
     return (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
            (size_t)(partition_size / kBlock) * 4;
   }
 };
 
+// Merge the partitions of (sequence s, head h) by log-sum-exp, in partition
+// order, and write the normalised output.  Lanes < CPR each own one 16-byte
+// output chunk.  Partials are read with .cg loads (L2), since other CTAs
+// wrote them during this launch.
+template <typename T, int D>
+__device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t sh, int np, int lane) {
+  using C = Chunk<T>;
+  constexpr int VEC = C::N;
+  constexpr int CPR = D / VEC;
+  if (lane >= CPR) return;
+  const float2* ml = a.part_ml + sh * a.max_parts;
+  float M = -INFINITY;
+  for (int p = 0; p < np; ++p) M = fmaxf(M, __ldcg(&ml[p]).x);
+  float den = 0.f;
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  const float* base = a.part_acc + sh * a.max_parts * D + lane * VEC;
+#pragma unroll 4
+  for (int p = 0; p < np; ++p) {
+    const float2 v = __ldcg(&ml[p]);
+    const float w = exp2f(v.x - M);
+    den = fmaf(v.y, w, den);
+    const float4* src = reinterpret_cast<const float4*>(base + (int64_t)p * D);
+#pragma unroll
+    for (int e = 0; e < VEC; e += 4) {
+      const float4 x = __ldcg(src + e / 4);
+      acc[e] = fmaf(w, x.x, acc[e]);
+      acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
+      acc[e + 2] = fmaf(w, x.z, acc[e + 2]);
+      acc[e + 3] = fmaf(w, x.w, acc[e + 3]);
+    }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] *= inv;
+  reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D)[lane] = C::from_float(acc);
+}
+
+// The persistent partition kernel: CTAs pull (sequence, partition, head
+// group) items from the plan's queue; each warp streams one head of the item
+// through its own NSTAGE ring of bulk copies.
 template <typename T, int D, int WARPS, int NSTAGE>
 __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) {
   using Cfg = DecodeConfig<T, D, WARPS, NSTAGE>;
   using C = Chunk<T>;
   constexpr int VEC = Cfg::VEC, CPR = Cfg::CPR, RPI = Cfg::RPI, NCH = Cfg::NCH;
   constexpr int TILE = Cfg::TILE;
-
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * NSTAGE * Cfg::STAGE_BYTES);
   int32_t* tbl = reinterpret_cast<int32_t*>(bars + WARPS * NSTAGE);
   __shared__ int32_t s_item;
   __shared__ int32_t s_abort;
+  __shared__ int32_t s_merge;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int H = a.heads;
   const int PS = a.partition_size;
-
   if (threadIdx.x == 0) {
     for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
@@ -190,11 +242,9 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
   const int32_t num_items = a.plan->num_items;
   __syncthreads();
-
   uint32_t fills = 0;  // stage fills this warp has consumed so far (drives ring slot + parity)
   uint8_t* my_stages = stages + warp * NSTAGE * Cfg::STAGE_BYTES;
   uint64_t* my_bars = bars + warp * NSTAGE;
-
   for (;;) {
     if (threadIdx.x == 0) {
       s_item = next;
@@ -203,35 +253,34 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
     __syncthreads();
     const int item = s_item;
     if (item >= num_items || s_abort) break;
-
     const int2 pr = a.pairs[item / a.head_groups];
     const int g = item % a.head_groups;
     const int s = pr.x, p = pr.y;
     const int L = a.lens[s];
-    const bool split = a.nparts[s] > 1;
+    const int np = a.nparts[s];
+    const bool split = np > 1;
     const int tok0 = p * PS;
     const int ntok = max(0, min(L, tok0 + PS) - tok0);
     const int nblk = (ntok + kBlock - 1) / kBlock;
     const int blk0 = tok0 / kBlock;
+    // the item holding the sequence's last token appends the new one (fused mode)
+    const bool append = a.k_new != nullptr && L > 0 && p == np - 1;
+    const int new_row = (L - 1) % kBlock;  // in-block offset of the appended token
 
     // block-table slice of this partition, bounds-checked once
     for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
       int32_t b = a.block_tables[(int64_t)s * a.max_blocks_per_seq + blk0 + i];
-      if (b < 0 || b >= a.num_blocks) {
-        atomicOr(a.err, PA_DEVERR_BLOCK_ID);
-        b = 0;
-      }
+      if (b < 0 || b >= a.num_blocks) { atomicOr(a.err, PA_DEVERR_BLOCK_ID); b = 0; }
       tbl[i] = b;
     }
     __syncthreads();
-
     const int h = g * WARPS + warp;
     if (h < H) {
       const int c = lane % CPR;  // this lane's chunk within a token row
+      const int64_t sh = (int64_t)s * H + h;
       float qf[VEC];
       {
-        const uint4 u =
-            reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + ((int64_t)s * H + h) * D)[c];
+        const uint4 u = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + sh * D)[c];
         C::to_float(u, qf);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) qf[e] *= a.scale_log2;
@@ -240,7 +289,6 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
       float acc[VEC];
 #pragma unroll
       for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-
       const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)h * TILE;
       const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)h * TILE;
       const int64_t block_bytes = (int64_t)H * TILE;
@@ -253,7 +301,6 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         bulk_copy_g2s(smem_addr(dst), kbase + off, TILE, bar);
         bulk_copy_g2s(smem_addr(dst + TILE), vbase + off, TILE, bar);
       };
-
       const uint32_t k0 = fills;
       if (lane == 0) {
         fence_proxy_async_shared();  // the previous item's reads of these stages are done
@@ -267,14 +314,24 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         const uint32_t k = k0 + i;
         const int st = k % NSTAGE;
         const bool landed = mbar_wait_bounded(smem_addr(&my_bars[st]), (k / NSTAGE) & 1u);
-        if (!__all_sync(kFullMask, landed)) {
-          ok = false;
-          break;
-        }
-        const uint4* kt = reinterpret_cast<const uint4*>(my_stages + st * Cfg::STAGE_BYTES);
-        const uint4* vt = kt + TILE / 16;
+        if (!__all_sync(kFullMask, landed)) { ok = false; break; }
+        uint4* kt = reinterpret_cast<uint4*>(my_stages + st * Cfg::STAGE_BYTES);
+        uint4* vt = kt + TILE / 16;
         const int valid = min(kBlock, ntok - i * kBlock);
-
+        if (append && i == nblk - 1) {
+          // fused reshape_and_cache: the new token's row goes to the pool and
+          // replaces the stale row of the staged tile
+          if (lane < CPR) {
+            const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + sh * D)[lane];
+            const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + sh * D)[lane];
+            kt[new_row * CPR + lane] = kn;
+            vt[new_row * CPR + lane] = vn;
+            const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * (TILE / kBlock);
+            reinterpret_cast<uint4*>(const_cast<char*>(kbase) + row_off)[lane] = kn;
+            reinterpret_cast<uint4*>(const_cast<char*>(vbase) + row_off)[lane] = vn;
+          }
+          __syncwarp();
+        }
         float part[NCH];
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
@@ -288,7 +345,6 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         halve<CPR / 2, NCH>(part, lane);
         float sc = part[0] + __shfl_xor_sync(kFullMask, part[0], 1);
         if (my_row >= valid) sc = -INFINITY;
-
         float bmax = sc;
 #pragma unroll
         for (int m = 2; m < 32; m <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFullMask, bmax, m));
@@ -302,7 +358,6 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         m_run = m_new;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] *= alpha;
-
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
           const float pj = __shfl_sync(kFullMask, pw, (lane / CPR) * CPR + 2 * j);
@@ -313,17 +368,11 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pj, vf[e], acc[e]);
         }
         __syncwarp();
-        if (lane == 0 && i + NSTAGE < nblk) {
-          fence_proxy_async_shared();
-          issue(k + NSTAGE, i + NSTAGE);
-        }
+        if (lane == 0 && i + NSTAGE < nblk) { fence_proxy_async_shared(); issue(k + NSTAGE, i + NSTAGE); }
       }
       if (!ok) {
         // give up on this item: report, let the copies already issued land, stop the CTA
-        if (lane == 0) {
-          atomicOr(a.err, PA_DEVERR_TIMEOUT);
-          s_abort = 1;
-        }
+        if (lane == 0) { atomicOr(a.err, PA_DEVERR_TIMEOUT); s_abort = 1; }
         const int issued = min(nblk, i + NSTAGE);
         for (int j = i; j < issued; ++j) {
           const uint32_t k = k0 + j;
@@ -338,7 +387,6 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(kFullMask, acc[e], m);
         }
         if (lane < CPR) {
-          const int64_t sh = (int64_t)s * H + h;
           if (!split) {
             float o[VEC];
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -348,67 +396,35 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           } else {
             float4* dst = reinterpret_cast<float4*>(a.part_acc + (sh * a.max_parts + p) * D + c * VEC);
 #pragma unroll
-            for (int e = 0; e < VEC; e += 4)
-              dst[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            for (int e = 0; e < VEC; e += 4) dst[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
             if (lane == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
           }
         }
       }
     }
+    if (split) {
+      // count this partition in; the last of the sequence's partitions merges.
+      // The barrier orders every warp's partial stores before thread 0's
+      // gpu-scope fence, which publishes them before the arrival count.
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
+        __threadfence();
+        const int arrived = atomicAdd(cnt, 1) + 1;
+        s_merge = arrived == np && !s_abort;
+        if (arrived == np) *cnt = 0;  // re-arm for the next launch on this plan
+      }
+      __syncthreads();
+      if (s_merge && h < H) { __threadfence(); merge_partitions<T, D>(a, (int64_t)s * H + h, np, lane); }
+    }
     __syncthreads();
   }
-
   // the last CTA out re-arms the queue so the plan can be reused
   if (threadIdx.x == 0) {
     __threadfence();
     const int done = atomicAdd(&a.plan->done_counter, 1);
-    if (done == (int)gridDim.x - 1) {
-      a.plan->work_counter = 0;
-      a.plan->done_counter = 0;
-      __threadfence();
-    }
+    if (done == (int)gridDim.x - 1) { a.plan->work_counter = 0; a.plan->done_counter = 0; __threadfence(); }
   }
-}
-
-// ---- split-K merge: one warp per (sequence, head) -----------------------------------
-
-template <typename T, int D>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(DecodeArgs a) {
-  using C = Chunk<T>;
-  constexpr int VEC = C::N;
-  constexpr int CPR = D / VEC;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t sh = (int64_t)blockIdx.x * 4 + warp;
-  if (sh >= (int64_t)a.num_seqs * a.heads) return;
-  const int s = (int)(sh / a.heads);
-  const int np = a.nparts[s];
-  if (np <= 1 || lane >= CPR) return;
-  const float2* ml = a.part_ml + sh * a.max_parts;
-  float M = -INFINITY;
-  for (int p = 0; p < np; ++p) M = fmaxf(M, ml[p].x);
-  float den = 0.f;
-  float acc[VEC];
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-  const float* base = a.part_acc + sh * a.max_parts * D + lane * VEC;
-  for (int p = 0; p < np; ++p) {
-    const float2 v = ml[p];
-    const float w = exp2f(v.x - M);
-    den = fmaf(v.y, w, den);
-    const float4* src = reinterpret_cast<const float4*>(base + (int64_t)p * D);
-#pragma unroll
-    for (int e = 0; e < VEC; e += 4) {
-      const float4 x = src[e / 4];
-      acc[e] = fmaf(w, x.x, acc[e]);
-      acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
-      acc[e + 2] = fmaf(w, x.z, acc[e + 2]);
-      acc[e + 3] = fmaf(w, x.w, acc[e + 3]);
-    }
-  }
-  const float inv = 1.f / den;
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) acc[e] *= inv;
-  reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D)[lane] = C::from_float(acc);
 }
 
 }  // namespace pa

@@ -21,15 +21,23 @@ __device__ uint32_t g_device_errors;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDecodeWarps = 4;   // heads per CTA (one warp each)
-constexpr int kDecodeStages = 3;  // per-warp ring depth
-constexpr int kDefaultPartition = 256;
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;    // heads per CTA (one warp each)
+constexpr int kDecodeStages = PA_DECODE_STAGES;  // per-warp ring depth
+constexpr int kMinAutoPartition = 256;    // smallest partition the automatic choice makes
+constexpr int kFullBatchPartition = 512;  // partition when the batch alone fills the GPU
 constexpr int kMaxPartition = 4096;
 
 struct DeviceState {
   bool ready = false;
   uint32_t* err = nullptr;  // device address of g_device_errors
   int num_sms = 0;
+  int decode_ctas_per_sm = 1;  // resident decode CTAs per SM (fp16, head_dim 128 kernel)
 };
 
 std::mutex g_mutex;
@@ -41,14 +49,28 @@ pa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(PA_ERR_CUDA, buf);
 }
 
+// Ring depth for a tile size: kDecodeStages, reduced until the CTA's stages
+// fit the 227 KB a CTA may use (fp32 tiles at head_dim 128 are 8 KB).
+constexpr int stages_for(int tile_bytes) {
+  int s = kDecodeStages;
+  while (s > 1 && kDecodeWarps * s * 2 * tile_bytes + 4096 > 227 * 1024) --s;
+  return s;
+}
+
 template <typename T, int D>
-using DecodeKernelCfg = DecodeConfig<T, D, kDecodeWarps, kDecodeStages>;
+using DecodeKernelCfg =
+    DecodeConfig<T, D, kDecodeWarps, stages_for(kBlock * D * (int)sizeof(T))>;
+
+template <typename T, int D>
+constexpr auto decode_kernel_ptr() {
+  return paged_decode_kernel<T, D, kDecodeWarps, stages_for(kBlock * D * (int)sizeof(T))>;
+}
 
 template <typename T, int D>
 cudaError_t set_decode_attrs() {
   const size_t smem = DecodeKernelCfg<T, D>::smem_bytes(kMaxPartition);
-  return cudaFuncSetAttribute(paged_decode_kernel<T, D, kDecodeWarps, kDecodeStages>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return cudaFuncSetAttribute(decode_kernel_ptr<T, D>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem);
 }
 
 // Once per device, with that device current: resolve the error word's device
@@ -72,6 +94,12 @@ pa_status device_state(DeviceState** out) {
                            set_decode_attrs<__nv_bfloat16, 64>(), set_decode_attrs<__nv_bfloat16, 128>()};
     for (cudaError_t a : attrs)
       if (a != cudaSuccess) return cuda_fail(a, "cudaFuncSetAttribute");
+    using Cfg = DecodeKernelCfg<__half, 128>;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&st.decode_ctas_per_sm,
+                                                      decode_kernel_ptr<__half, 128>(),
+                                                      Cfg::THREADS, Cfg::smem_bytes(2048));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    st.decode_ctas_per_sm = std::max(1, st.decode_ctas_per_sm);
     st.ready = true;
   }
   *out = &st;
@@ -93,7 +121,8 @@ pa_status check_pool(const pa_pool* pool) {
 }
 
 struct WorkspaceLayout {
-  size_t header = 0, lens = 0, nparts = 0, pairs = 0, part_ml = 0, part_acc = 0, total = 0;
+  size_t header = 0, lens = 0, nparts = 0, merge_cnt = 0, pairs = 0, part_ml = 0, part_acc = 0,
+         total = 0;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -107,6 +136,8 @@ WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D) {
   off = align256(off + S * 4);
   w.nparts = off;
   off = align256(off + S * 4);
+  w.merge_cnt = off;
+  off = align256(off + S * ((H + kDecodeWarps - 1) / kDecodeWarps) * 4);
   w.pairs = off;
   off = align256(off + S * max_parts * 8);
   w.part_ml = off;
@@ -117,8 +148,21 @@ WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D) {
   return w;
 }
 
-int resolve_partition(int32_t partition_size) {
-  return partition_size == 0 ? kDefaultPartition : partition_size;
+int round_up16(int64_t x) { return (int)std::min<int64_t>(kMaxPartition, (x + 15) / 16 * 16); }
+
+// Automatic partition size.  Every work item pays a pipeline ramp and a
+// split costs partial results and a merge, while one long item is streamed
+// by a single CTA at a fraction of the chip's bandwidth and can become the
+// critical path.  Measured on B200: when (sequences x head groups) already
+// gives two items per resident CTA, 512-token partitions are best; with few
+// sequences, aim for about four items per resident CTA (never below 256).
+int auto_partition(int num_seqs, int head_groups, int max_context_len, int slots) {
+  const int64_t whole = (int64_t)num_seqs * head_groups;
+  const int64_t maxL = std::max(16, max_context_len);
+  if (whole >= 2LL * slots) return std::min(kFullBatchPartition, round_up16(maxL));
+  const int64_t want_parts = (4LL * slots + whole - 1) / std::max<int64_t>(whole, 1);
+  const int64_t ps = (maxL + want_parts - 1) / want_parts;
+  return std::max(kMinAutoPartition, round_up16(ps));
 }
 
 int resolve_max_context(const pa_pool* pool, int32_t max_blocks_per_seq, int32_t max_context_len) {
@@ -130,7 +174,7 @@ int resolve_max_context(const pa_pool* pool, int32_t max_blocks_per_seq, int32_t
 template <typename T, int D>
 cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
   using Cfg = DecodeKernelCfg<T, D>;
-  auto kernel = paged_decode_kernel<T, D, kDecodeWarps, kDecodeStages>;
+  auto kernel = decode_kernel_ptr<T, D>();
   const size_t smem = Cfg::smem_bytes(a.partition_size);
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Cfg::THREADS, smem);
@@ -139,14 +183,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStrea
   const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
   kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int64_t pairs = (int64_t)a.num_seqs * a.heads;
-  if (a.max_parts > 1) {
-    paged_decode_merge_kernel<T, D><<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(a);
-    e = cudaGetLastError();
-  }
-  return e;
+  return cudaGetLastError();
 }
 
 // One warp waits on a barrier that expects two arrivals but gets one.
@@ -224,7 +261,8 @@ pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
   if (!bytes) return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bytes is null");
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
     return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bad size");
-  const int ps = resolve_partition(partition_size);
+  // partition_size 0: the automatic choice is never below kMinAutoPartition
+  const int ps = partition_size == 0 ? kMinAutoPartition : partition_size;
   if (ps < kBlock || ps % kBlock != 0 || ps > kMaxPartition)
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
@@ -246,15 +284,20 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   if (st != PA_OK) return st;
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
     return fail(PA_ERR_INVALID_ARG, "decode: bad size");
-  const int ps = resolve_partition(partition_size);
-  if (ps < kBlock || ps % kBlock != 0 || ps > kMaxPartition)
+  if (partition_size != 0 &&
+      (partition_size < kBlock || partition_size % kBlock != 0 || partition_size > kMaxPartition))
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
+  if ((st = device_state(dev)) != PA_OK) return st;
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
+  const int head_groups = (pool->heads + kDecodeWarps - 1) / kDecodeWarps;
+  const int ps = partition_size != 0
+                     ? partition_size
+                     : auto_partition(num_seqs, head_groups, maxL,
+                                      (*dev)->num_sms * (*dev)->decode_ctas_per_sm);
   const int max_parts = std::max(1, (maxL + ps - 1) / ps);
   const WorkspaceLayout w = layout_for(num_seqs, pool->heads, max_parts, pool->head_dim);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(PA_ERR_WORKSPACE, "decode: workspace missing, not 256-byte aligned or too small");
-  if ((st = device_state(dev)) != PA_OK) return st;
   char* ws = static_cast<char*>(workspace);
   *a = DecodeArgs{};
   a->plan = reinterpret_cast<PlanHeader*>(ws + w.header);
@@ -263,6 +306,7 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   a->pairs = reinterpret_cast<int2*>(ws + w.pairs);
   a->part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
   a->part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+  a->merge_cnt = reinterpret_cast<int32_t*>(ws + w.merge_cnt);
   a->err = (*dev)->err;
   a->num_blocks = pool->num_blocks;
   a->max_blocks_per_seq = max_blocks_per_seq;
@@ -374,6 +418,50 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = launch_plan(a, s)) != PA_OK) return st;
   return launch_run(pool, a, *dev, s);
+}
+
+pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
+                                             const void* k_new, const void* v_new, void* k_pool,
+                                             void* v_pool, const int32_t* block_tables,
+                                             int32_t max_blocks_per_seq, int32_t num_seqs,
+                                             int32_t max_context_len, float scale, void* out,
+                                             void* workspace, size_t workspace_bytes,
+                                             int32_t partition_size, void* stream) {
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode append: num_seqs < 0");
+  if (num_seqs == 0) return check_pool(pool);
+  pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
+  if (st != PA_OK) return st;
+  if (!k_new || !v_new) return fail(PA_ERR_INVALID_ARG, "decode append: k_new/v_new is null");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(PA_ERR_INVALID_ARG, "decode append: k_new/v_new must be 16-byte aligned");
+  DecodeArgs a;
+  DeviceState* dev;
+  st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+                      workspace, workspace_bytes, &a, &dev);
+  if (st != PA_OK) return st;
+  set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  return launch_run(pool, a, *dev, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_append_attention(const pa_pool* pool, const void* q, const void* k_new,
+                                     const void* v_new, void* k_pool, void* v_pool,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t max_context_len, float scale, void* out,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t partition_size, void* stream) {
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode append: num_seqs < 0");
+  if (num_seqs == 0) return check_pool(pool);
+  pa_status st = pa_decode_plan(pool, context_lens, num_seqs, max_blocks_per_seq,
+                                max_context_len, partition_size, workspace, workspace_bytes,
+                                stream);
+  if (st != PA_OK) return st;
+  return pa_decode_append_attention_planned(pool, q, k_new, v_new, k_pool, v_pool, block_tables,
+                                            max_blocks_per_seq, num_seqs, max_context_len, scale,
+                                            out, workspace, workspace_bytes, partition_size,
+                                            stream);
 }
 
 pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,

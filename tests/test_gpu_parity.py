@@ -306,3 +306,58 @@ def test_plan_once_run_many_layers_matches_single_calls():
         ref = oracle.decode_attention(host(q), host(kp), host(vp), case["block_tables"],
                                       case["context_lens"], case["scale"])
         assert_parity(got, ref, "planned layer")
+
+
+# ---- fused append + attend ------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,head_dim,partition_size", [(np.float16, 128, 0), (np.float16, 64, 32),
+                                                           (np.float32, 128, 16), (np.float32, 64, 0)])
+def test_fused_append_equals_cache_then_decode(dtype, head_dim, partition_size):
+    """One launch that writes the new token and attends must leave the same
+    pool bits and produce the same output bits as reshape_and_cache followed
+    by decode, and match the oracle."""
+    lens = [0, 1, 2, 16, 17, 32, 33, 255, 256, 257, 1000, 2048, 5]
+    case = syn.decode_case(31, lens, 6, head_dim, dtype, max_blocks=130)
+    ref_out, ref_k, ref_v = gpu_append_and_decode(case, partition_size=partition_size)
+    q, kp, vp = dev(case["q"]), dev(case["k_pool"]), dev(case["v_pool"])
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    NB = kp.shape[0]
+    pool = pa.pa_pool_create(NB, 16, 6, head_dim, q.dtype)
+    out = torch.empty_like(q)
+    ws = workspace_for(pool, len(lens), bt.shape[1], 0, partition_size)
+    pa.pa_decode_append_attention(pool, q, dev(case["k_new"]), dev(case["v_new"]), kp, vp, bt, cl,
+                                  case["scale"], out, ws, partition_size=partition_size)
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(bits_t(kp), bits_t(ref_k)) and torch.equal(bits_t(vp), bits_t(ref_v))
+    assert torch.equal(out, ref_out)
+    want, _, _ = oracle_append_and_decode(case)
+    assert_parity(out, want, "fused append")
+
+
+def bits_t(t):
+    return t.view(torch.int16 if t.element_size() == 2 else torch.int32)
+
+
+def test_fused_append_planned_over_layers():
+    case = syn.single_layer_case(seed=8, num_seqs=32)
+    NB, H, BS, D = case["k_pool"].shape
+    pool = pa.pa_pool_create(NB, BS, H, D, torch.float16)
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    ws = workspace_for(pool, 32, bt.shape[1])
+    pa.pa_decode_plan(pool, cl, bt.shape[1], ws)
+    rng = np.random.default_rng(12)
+    for layer in range(3):
+        kp_h = rng.standard_normal(case["k_pool"].shape).astype(np.float16)
+        vp_h = rng.standard_normal(case["k_pool"].shape).astype(np.float16)
+        q_h = rng.standard_normal(case["q"].shape).astype(np.float16)
+        kn_h = rng.standard_normal(case["q"].shape).astype(np.float16)
+        vn_h = rng.standard_normal(case["q"].shape).astype(np.float16)
+        kp, vp, q = dev(kp_h), dev(vp_h), dev(q_h)
+        out = torch.empty_like(q)
+        pa.pa_decode_append_attention_planned(pool, q, dev(kn_h), dev(vn_h), kp, vp, bt,
+                                              case["scale"], out, ws)
+        assert pa.pa_device_errors() == 0
+        layer_case = dict(case, k_pool=kp_h, v_pool=vp_h, q=q_h, k_new=kn_h, v_new=vn_h)
+        want, wk, wv = oracle_append_and_decode(layer_case)
+        assert np.array_equal(bits(kp), bits(wk)) and np.array_equal(bits(vp), bits(wv))
+        assert_parity(out, want, f"fused planned layer {layer}")
