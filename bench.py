@@ -93,8 +93,8 @@ def committed_traffic():
         return None
     vals = {}
     for line in text.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
+        if ": " in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(": ", 1)
             vals[k.strip()] = v.strip().strip("`")
     if vals.get("decode.cuh sha256[:16]") != decode_source_hash():
         return None
