@@ -18,7 +18,9 @@
  *   k_pool, v_pool   [num_blocks][heads][block_size][head_dim], dtype elements,
  *                    16-byte aligned base.  Physical slot of a token =
  *                    block_id * block_size + in-block offset.
- *   q, out           [num_seqs][heads][head_dim], same dtype as the pool.
+ *   q, out           [num_seqs][heads * q_per_kv][head_dim], same dtype as
+ *                    the pool (q_per_kv = 1 unless pa_pool_set_query_heads).
+ *   k_new, v_new of the fused append: [num_seqs][heads][head_dim].
  *   k_new, v_new     [num_tokens][heads][head_dim], same dtype as the pool.
  *   block_tables     int32 [num_seqs][max_blocks_per_seq]; entries past a
  *                    sequence's last block are never read.
@@ -76,7 +78,7 @@ typedef struct pa_pool {
   int32_t head_dim;
   int32_t dtype;       /* pa_dtype */
   int32_t elem_bytes;
-  int32_t reserved;
+  int32_t q_per_kv;     /* query heads per KV head: 1 (MHA), 2, 4 or 8 (GQA/MQA) */
   int64_t token_stride; /* elements between consecutive slots of a block: head_dim */
   int64_t head_stride;  /* elements between heads of a block: block_size * head_dim */
   int64_t block_stride; /* elements between blocks: heads * block_size * head_dim */
@@ -92,6 +94,16 @@ typedef struct pa_pool {
  */
 pa_status pa_pool_create(int64_t num_blocks, int32_t block_size, int32_t heads,
                          int32_t head_dim, int32_t dtype, pa_pool* out);
+
+/*
+ * Grouped-query attention (no counterpart on the pages, which use one query
+ * head per KV head): declare that q and out carry num_q_heads heads, a
+ * multiple (1, 2, 4 or 8) of the pool's KV heads.  Query head h reads KV
+ * head h / (num_q_heads / heads).  The pool itself (and reshape_and_cache,
+ * copy_blocks, k_new and v_new) keeps the KV head count.  The KV tile is read
+ * once per KV head and shared by its query heads.
+ */
+pa_status pa_pool_set_query_heads(pa_pool* pool, int32_t num_q_heads);
 
 /*
  * Write each new token's K and V rows into the slot slot_mapping names:

@@ -45,7 +45,7 @@ class pa_pool(ctypes.Structure):
         ("head_dim", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
         ("elem_bytes", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("q_per_kv", ctypes.c_int32),
         ("token_stride", ctypes.c_int64),
         ("head_stride", ctypes.c_int64),
         ("block_stride", ctypes.c_int64),
@@ -68,6 +68,7 @@ def lib():
         P = ctypes.POINTER
         sigs = {
             "pa_pool_create": [i64, i32, i32, i32, i32, P(pa_pool)],
+            "pa_pool_set_query_heads": [P(pa_pool), i32],
             "pa_reshape_and_cache": [P(pa_pool), vp, vp, vp, i32, vp, vp, vp],
             "pa_decode_workspace_bytes": [P(pa_pool), i32, i32, i32, i32, P(sz)],
             "pa_decode_attention": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, i32, ctypes.c_float,
@@ -162,6 +163,16 @@ def pa_pool_create(num_blocks: int, block_size: int, heads: int, head_dim: int, 
     return p
 
 
+def pa_pool_set_query_heads(pool: pa_pool, num_q_heads: int) -> pa_pool:
+    """GQA/MQA: q and out carry num_q_heads (1, 2, 4 or 8 per KV head)."""
+    _check(lib().pa_pool_set_query_heads(ctypes.byref(pool), num_q_heads))
+    return pool
+
+
+def _q_heads(pool: pa_pool) -> int:
+    return pool.heads * pool.q_per_kv
+
+
 def _pool_torch_dtype(pool: pa_pool):
     torch = _torch()
     return {PA_F32: torch.float32, PA_F16: torch.float16, PA_BF16: torch.bfloat16}[pool.dtype]
@@ -200,8 +211,8 @@ def pa_decode_attention(pool, q, k_pool, v_pool, block_tables, context_lens, sca
                         workspace, max_context_len=0, partition_size=0, stream=None):
     torch = _torch()
     S = q.shape[0]
-    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
     if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
     dt = _pool_torch_dtype(pool)
@@ -228,8 +239,8 @@ def pa_decode_attention_planned(pool, q, k_pool, v_pool, block_tables, scale, ou
                                 max_context_len=0, partition_size=0, stream=None):
     torch = _torch()
     S = q.shape[0]
-    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
     if block_tables.dim() != 2 or block_tables.shape[0] != S:
         raise ValueError("block_tables must be [num_seqs, max_blocks]")
     dt = _pool_torch_dtype(pool)
@@ -248,10 +259,11 @@ def pa_decode_append_attention(pool, q, k_new, v_new, k_pool, v_pool, block_tabl
     decode attention in one launch; k_new/v_new are [num_seqs, heads, head_dim]."""
     torch = _torch()
     S = q.shape[0]
-    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
-    if tuple(k_new.shape) != tuple(q.shape) or tuple(v_new.shape) != tuple(q.shape):
-        raise ValueError("k_new and v_new must be [num_seqs, heads, head_dim]")
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
+    kv_shape = (S, pool.heads, pool.head_dim)
+    if tuple(k_new.shape) != kv_shape or tuple(v_new.shape) != kv_shape:
+        raise ValueError("k_new and v_new must be [num_seqs, KV heads, head_dim]")
     if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
     dt = _pool_torch_dtype(pool)
@@ -270,10 +282,11 @@ def pa_decode_append_attention_planned(pool, q, k_new, v_new, k_pool, v_pool, bl
                                        stream=None):
     torch = _torch()
     S = q.shape[0]
-    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
-    if tuple(k_new.shape) != tuple(q.shape) or tuple(v_new.shape) != tuple(q.shape):
-        raise ValueError("k_new and v_new must be [num_seqs, heads, head_dim]")
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
+    kv_shape = (S, pool.heads, pool.head_dim)
+    if tuple(k_new.shape) != kv_shape or tuple(v_new.shape) != kv_shape:
+        raise ValueError("k_new and v_new must be [num_seqs, KV heads, head_dim]")
     if block_tables.dim() != 2 or block_tables.shape[0] != S:
         raise ValueError("block_tables must be [num_seqs, max_blocks]")
     dt = _pool_torch_dtype(pool)
@@ -297,8 +310,8 @@ def pa_decode_attention_static(pool, q, k_pool, v_pool, block_tables, context_le
     the GPU; the first call on a device must come before any stream capture."""
     torch = _torch()
     S = q.shape[0]
-    if tuple(q.shape) != (S, pool.heads, pool.head_dim) or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("q and out must be [num_seqs, heads, head_dim]")
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
     if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
     dt = _pool_torch_dtype(pool)

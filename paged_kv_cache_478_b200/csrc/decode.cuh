@@ -75,8 +75,9 @@ struct DecodeArgs {
   int64_t num_blocks;
   int32_t max_blocks_per_seq;
   int32_t num_seqs;
-  int32_t heads;
-  int32_t head_groups;
+  int32_t heads;        // KV heads in the pool
+  int32_t q_per_kv;     // query heads per KV head (1 = MHA; GQA/MQA otherwise)
+  int32_t head_groups;  // work items per (sequence, partition)
   int32_t partition_size;
   int32_t max_parts;
   int32_t max_context_len;
@@ -155,7 +156,9 @@ __device__ __forceinline__ void halve(float* v, int lane) {
 
 // ---- the partition kernel -----------------------------------------------------------
 
-template <typename T, int D, int WARPS, int NSTAGE>
+// G = query heads per KV head that share one ring: the G warps of a ring
+// read the same staged (block, KV head) tile, each with its own query head.
+template <typename T, int D, int WARPS, int NSTAGE, int G>
 struct DecodeConfig {
   static constexpr int VEC = Chunk<T>::N;      // elements per 16-byte chunk
   static constexpr int CPR = D / VEC;          // chunks (= lanes) per token row
@@ -164,14 +167,45 @@ struct DecodeConfig {
   static constexpr int TILE = kBlock * D * (int)sizeof(T);  // one (block, head) tile
   static constexpr int STAGE_BYTES = 2 * TILE;              // K tile + V tile
   static constexpr int THREADS = WARPS * 32;
+  static constexpr int RINGS = WARPS / G;      // KV heads per work item
   static_assert(CPR >= 2 && CPR <= 32 && 32 % CPR == 0, "head_dim / dtype not supported");
   static_assert(NCH * 2 == CPR, "lane mapping");
+  static_assert(WARPS % G == 0 && RINGS >= 1, "a ring's warps must fit the CTA");
   // stage rings + one mbarrier per stage + the item's block-table slice
   static size_t smem_bytes(int partition_size) {
-    return (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
+    return (size_t)RINGS * NSTAGE * STAGE_BYTES + (size_t)RINGS * NSTAGE * 8 +
            (size_t)(partition_size / kBlock) * 4;
   }
 };
+
+// Barrier over the G warps of ring r (named barrier 1 + r); returns whether
+// every participating thread passed ok.  With G == 1 it is a warp vote.
+template <int G>
+__device__ __forceinline__ bool ring_vote(int r, bool ok) {
+  if constexpr (G == 1) {
+    return __all_sync(kFullMask, ok);
+  } else {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)ok), "r"(1 + r), "r"(G * 32)
+        : "memory");
+    return res != 0;
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void ring_sync(int r) {
+  if constexpr (G == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + r), "r"(G * 32) : "memory");
+  }
+}
 
 // Merge the partitions of (sequence s, head h) by log-sum-exp, in partition
 // order, and write the normalised output.  Lanes < CPR each own one 16-byte
@@ -213,28 +247,34 @@ __device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t sh
 }
 
 // The persistent partition kernel: CTAs pull (sequence, partition, head
-// group) items from the plan's queue; each warp streams one head of the item
-// through its own NSTAGE ring of bulk copies.
-template <typename T, int D, int WARPS, int NSTAGE>
+// group) items from the plan's queue.  Each ring of G warps streams one KV
+// head of the item through NSTAGE stages of bulk copies; each warp of the
+// ring attends with its own query head (G == 1: one warp per head).
+template <typename T, int D, int WARPS, int NSTAGE, int G>
 __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) {
-  using Cfg = DecodeConfig<T, D, WARPS, NSTAGE>;
+  using Cfg = DecodeConfig<T, D, WARPS, NSTAGE, G>;
   using C = Chunk<T>;
   constexpr int VEC = Cfg::VEC, CPR = Cfg::CPR, RPI = Cfg::RPI, NCH = Cfg::NCH;
-  constexpr int TILE = Cfg::TILE;
+  constexpr int TILE = Cfg::TILE, RINGS = Cfg::RINGS;
+
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * NSTAGE * Cfg::STAGE_BYTES);
-  int32_t* tbl = reinterpret_cast<int32_t*>(bars + WARPS * NSTAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RINGS * NSTAGE * Cfg::STAGE_BYTES);
+  int32_t* tbl = reinterpret_cast<int32_t*>(bars + RINGS * NSTAGE);
   __shared__ int32_t s_item;
   __shared__ int32_t s_abort;
   __shared__ int32_t s_merge;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int H = a.heads;
+  const int ring = warp / G;            // which KV head of the item this warp serves
+  const bool leader = (warp % G) == 0;  // lane 0 of the leader warp issues the ring's copies
+  const int HK = a.heads;               // KV heads
+  const int HQ = a.heads * G;           // query heads
   const int PS = a.partition_size;
+
   if (threadIdx.x == 0) {
-    for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    for (int i = 0; i < RINGS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
     s_abort = 0;
   }
@@ -242,9 +282,11 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
   const int32_t num_items = a.plan->num_items;
   __syncthreads();
-  uint32_t fills = 0;  // stage fills this warp has consumed so far (drives ring slot + parity)
-  uint8_t* my_stages = stages + warp * NSTAGE * Cfg::STAGE_BYTES;
-  uint64_t* my_bars = bars + warp * NSTAGE;
+
+  uint32_t fills = 0;  // stage fills this ring has consumed so far (drives ring slot + parity)
+  uint8_t* my_stages = stages + ring * NSTAGE * Cfg::STAGE_BYTES;
+  uint64_t* my_bars = bars + ring * NSTAGE;
+
   for (;;) {
     if (threadIdx.x == 0) {
       s_item = next;
@@ -253,6 +295,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
     __syncthreads();
     const int item = s_item;
     if (item >= num_items || s_abort) break;
+
     const int2 pr = a.pairs[item / a.head_groups];
     const int g = item % a.head_groups;
     const int s = pr.x, p = pr.y;
@@ -270,14 +313,19 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
     // block-table slice of this partition, bounds-checked once
     for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
       int32_t b = a.block_tables[(int64_t)s * a.max_blocks_per_seq + blk0 + i];
-      if (b < 0 || b >= a.num_blocks) { atomicOr(a.err, PA_DEVERR_BLOCK_ID); b = 0; }
+      if (b < 0 || b >= a.num_blocks) {
+        atomicOr(a.err, PA_DEVERR_BLOCK_ID);
+        b = 0;
+      }
       tbl[i] = b;
     }
     __syncthreads();
-    const int h = g * WARPS + warp;
-    if (h < H) {
+
+    const int kvh = g * RINGS + ring;          // KV head
+    const int hq = kvh * G + (warp % G);       // this warp's query head
+    if (kvh < HK) {
       const int c = lane % CPR;  // this lane's chunk within a token row
-      const int64_t sh = (int64_t)s * H + h;
+      const int64_t sh = (int64_t)s * HQ + hq;
       float qf[VEC];
       {
         const uint4 u = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + sh * D)[c];
@@ -289,9 +337,10 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
       float acc[VEC];
 #pragma unroll
       for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-      const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)h * TILE;
-      const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)h * TILE;
-      const int64_t block_bytes = (int64_t)H * TILE;
+
+      const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)kvh * TILE;
+      const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)kvh * TILE;
+      const int64_t block_bytes = (int64_t)HK * TILE;
       auto issue = [&](uint32_t k, int bi) {
         const int st = k % NSTAGE;
         const uint32_t bar = smem_addr(&my_bars[st]);
@@ -301,8 +350,9 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         bulk_copy_g2s(smem_addr(dst), kbase + off, TILE, bar);
         bulk_copy_g2s(smem_addr(dst + TILE), vbase + off, TILE, bar);
       };
+
       const uint32_t k0 = fills;
-      if (lane == 0) {
+      if (leader && lane == 0) {
         fence_proxy_async_shared();  // the previous item's reads of these stages are done
         for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
       }
@@ -314,16 +364,16 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         const uint32_t k = k0 + i;
         const int st = k % NSTAGE;
         const bool landed = mbar_wait_bounded(smem_addr(&my_bars[st]), (k / NSTAGE) & 1u);
-        if (!__all_sync(kFullMask, landed)) { ok = false; break; }
         uint4* kt = reinterpret_cast<uint4*>(my_stages + st * Cfg::STAGE_BYTES);
         uint4* vt = kt + TILE / 16;
         const int valid = min(kBlock, ntok - i * kBlock);
-        if (append && i == nblk - 1) {
+        if (append && i == nblk - 1 && leader && __all_sync(kFullMask, landed)) {
           // fused reshape_and_cache: the new token's row goes to the pool and
-          // replaces the stale row of the staged tile
+          // replaces the stale row of the staged tile (before the ring reads it)
           if (lane < CPR) {
-            const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + sh * D)[lane];
-            const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + sh * D)[lane];
+            const int64_t skv = (int64_t)s * HK + kvh;
+            const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + skv * D)[lane];
+            const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + skv * D)[lane];
             kt[new_row * CPR + lane] = kn;
             vt[new_row * CPR + lane] = vn;
             const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * (TILE / kBlock);
@@ -332,6 +382,11 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           }
           __syncwarp();
         }
+        if (!ring_vote<G>(ring, landed)) {  // the ring gives up together
+          ok = false;
+          break;
+        }
+
         float part[NCH];
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
@@ -345,6 +400,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         halve<CPR / 2, NCH>(part, lane);
         float sc = part[0] + __shfl_xor_sync(kFullMask, part[0], 1);
         if (my_row >= valid) sc = -INFINITY;
+
         float bmax = sc;
 #pragma unroll
         for (int m = 2; m < 32; m <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(kFullMask, bmax, m));
@@ -358,6 +414,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         m_run = m_new;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] *= alpha;
+
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
           const float pj = __shfl_sync(kFullMask, pw, (lane / CPR) * CPR + 2 * j);
@@ -367,12 +424,18 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
 #pragma unroll
           for (int e = 0; e < VEC; ++e) acc[e] = fmaf(pj, vf[e], acc[e]);
         }
-        __syncwarp();
-        if (lane == 0 && i + NSTAGE < nblk) { fence_proxy_async_shared(); issue(k + NSTAGE, i + NSTAGE); }
+        ring_sync<G>(ring);  // every warp of the ring is done with this stage
+        if (leader && lane == 0 && i + NSTAGE < nblk) {
+          fence_proxy_async_shared();
+          issue(k + NSTAGE, i + NSTAGE);
+        }
       }
       if (!ok) {
         // give up on this item: report, let the copies already issued land, stop the CTA
-        if (lane == 0) { atomicOr(a.err, PA_DEVERR_TIMEOUT); s_abort = 1; }
+        if (lane == 0) {
+          atomicOr(a.err, PA_DEVERR_TIMEOUT);
+          s_abort = 1;
+        }
         const int issued = min(nblk, i + NSTAGE);
         for (int j = i; j < issued; ++j) {
           const uint32_t k = k0 + j;
@@ -396,7 +459,8 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           } else {
             float4* dst = reinterpret_cast<float4*>(a.part_acc + (sh * a.max_parts + p) * D + c * VEC);
 #pragma unroll
-            for (int e = 0; e < VEC; e += 4) dst[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            for (int e = 0; e < VEC; e += 4)
+              dst[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
             if (lane == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
           }
         }
@@ -415,15 +479,23 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         if (arrived == np) *cnt = 0;  // re-arm for the next launch on this plan
       }
       __syncthreads();
-      if (s_merge && h < H) { __threadfence(); merge_partitions<T, D>(a, (int64_t)s * H + h, np, lane); }
+      if (s_merge && kvh < HK) {
+        __threadfence();
+        merge_partitions<T, D>(a, (int64_t)s * HQ + hq, np, lane);
+      }
     }
     __syncthreads();
   }
+
   // the last CTA out re-arms the queue so the plan can be reused
   if (threadIdx.x == 0) {
     __threadfence();
     const int done = atomicAdd(&a.plan->done_counter, 1);
-    if (done == (int)gridDim.x - 1) { a.plan->work_counter = 0; a.plan->done_counter = 0; __threadfence(); }
+    if (done == (int)gridDim.x - 1) {
+      a.plan->work_counter = 0;
+      a.plan->done_counter = 0;
+      __threadfence();
+    }
   }
 }
 

@@ -49,29 +49,49 @@ pa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(PA_ERR_CUDA, buf);
 }
 
-// Ring depth for a tile size: kDecodeStages, reduced until the CTA's stages
-// fit the 227 KB a CTA may use (fp32 tiles at head_dim 128 are 8 KB).
-constexpr int stages_for(int tile_bytes) {
-  int s = kDecodeStages;
-  while (s > 1 && kDecodeWarps * s * 2 * tile_bytes + 4096 > 227 * 1024) --s;
+// Warps per CTA for G query heads per KV head: G warps share one ring, and
+// a CTA keeps at least kDecodeWarps warps.
+constexpr int warps_for(int G) { return G > kDecodeWarps ? G : kDecodeWarps; }
+
+// Ring depth: the CTA keeps kDecodeWarps * kDecodeStages stages in flight
+// whatever the grouping (at most 8 per ring), reduced until the stages fit
+// the 227 KB a CTA may use (fp32 tiles at head_dim 128 are 8 KB).
+constexpr int stages_for(int tile_bytes, int G) {
+  const int rings = warps_for(G) / G;
+  int s = kDecodeWarps * kDecodeStages / rings;
+  if (s > 8) s = 8;
+  if (s < 1) s = 1;
+  while (s > 1 && rings * s * 2 * tile_bytes + 4096 > 227 * 1024) --s;
   return s;
 }
 
-template <typename T, int D>
+template <typename T, int D, int G>
 using DecodeKernelCfg =
-    DecodeConfig<T, D, kDecodeWarps, stages_for(kBlock * D * (int)sizeof(T))>;
+    DecodeConfig<T, D, warps_for(G), stages_for(kBlock * D * (int)sizeof(T), G), G>;
 
-template <typename T, int D>
+template <typename T, int D, int G>
 constexpr auto decode_kernel_ptr() {
-  return paged_decode_kernel<T, D, kDecodeWarps, stages_for(kBlock * D * (int)sizeof(T))>;
+  return paged_decode_kernel<T, D, warps_for(G), stages_for(kBlock * D * (int)sizeof(T), G), G>;
+}
+
+template <typename T, int D, int G>
+cudaError_t set_decode_attrs() {
+  const size_t smem = DecodeKernelCfg<T, D, G>::smem_bytes(kMaxPartition);
+  return cudaFuncSetAttribute(decode_kernel_ptr<T, D, G>(),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
 }
 
 template <typename T, int D>
-cudaError_t set_decode_attrs() {
-  const size_t smem = DecodeKernelCfg<T, D>::smem_bytes(kMaxPartition);
-  return cudaFuncSetAttribute(decode_kernel_ptr<T, D>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem);
+cudaError_t set_decode_attrs_all_groups() {
+  cudaError_t e = set_decode_attrs<T, D, 1>();
+  if (e == cudaSuccess) e = set_decode_attrs<T, D, 2>();
+  if (e == cudaSuccess) e = set_decode_attrs<T, D, 4>();
+  if (e == cudaSuccess) e = set_decode_attrs<T, D, 8>();
+  return e;
 }
+
+// KV heads one work item covers, for G query heads per KV head.
+int rings_for(int G) { return warps_for(G) / G; }
 
 // Once per device, with that device current: resolve the error word's device
 // address and raise the shared-memory limit of the decode kernels.
@@ -89,15 +109,18 @@ pa_status device_state(DeviceState** out) {
     st.err = static_cast<uint32_t*>(p);
     e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-    cudaError_t attrs[] = {set_decode_attrs<float, 64>(),          set_decode_attrs<float, 128>(),
-                           set_decode_attrs<__half, 64>(),         set_decode_attrs<__half, 128>(),
-                           set_decode_attrs<__nv_bfloat16, 64>(), set_decode_attrs<__nv_bfloat16, 128>()};
+    cudaError_t attrs[] = {set_decode_attrs_all_groups<float, 64>(),
+                           set_decode_attrs_all_groups<float, 128>(),
+                           set_decode_attrs_all_groups<__half, 64>(),
+                           set_decode_attrs_all_groups<__half, 128>(),
+                           set_decode_attrs_all_groups<__nv_bfloat16, 64>(),
+                           set_decode_attrs_all_groups<__nv_bfloat16, 128>()};
     for (cudaError_t a : attrs)
       if (a != cudaSuccess) return cuda_fail(a, "cudaFuncSetAttribute");
-    using Cfg = DecodeKernelCfg<__half, 128>;
+    using Cfg = DecodeKernelCfg<__half, 128, 1>;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&st.decode_ctas_per_sm,
-                                                      decode_kernel_ptr<__half, 128>(),
-                                                      Cfg::THREADS, Cfg::smem_bytes(2048));
+                                                      decode_kernel_ptr<__half, 128, 1>(),
+                                                      Cfg::THREADS, Cfg::smem_bytes(512));
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     st.decode_ctas_per_sm = std::max(1, st.decode_ctas_per_sm);
     st.ready = true;
@@ -114,6 +137,8 @@ pa_status check_pool(const pa_pool* pool) {
   if (pool->head_dim != 64 && pool->head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (pool->dtype < PA_F32 || pool->dtype > PA_BF16) return fail(PA_ERR_UNSUPPORTED, "unknown dtype");
+  if (pool->q_per_kv != 1 && pool->q_per_kv != 2 && pool->q_per_kv != 4 && pool->q_per_kv != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4 or 8");
   if (pool->num_blocks <= 0 || pool->heads <= 0) return fail(PA_ERR_INVALID_ARG, "empty pool");
   if (pool->num_blocks * pool->block_size > INT32_MAX)
     return fail(PA_ERR_INVALID_ARG, "num_blocks * block_size must fit int32");
@@ -127,7 +152,8 @@ struct WorkspaceLayout {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D) {
+// H = query heads (partials are per query head); G = query heads per KV head.
+WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D, int G) {
   WorkspaceLayout w;
   size_t off = 0;
   w.header = off;
@@ -137,7 +163,7 @@ WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D) {
   w.nparts = off;
   off = align256(off + S * 4);
   w.merge_cnt = off;
-  off = align256(off + S * ((H + kDecodeWarps - 1) / kDecodeWarps) * 4);
+  off = align256(off + S * ((H / G + rings_for(G) - 1) / rings_for(G)) * 4);
   w.pairs = off;
   off = align256(off + S * max_parts * 8);
   w.part_ml = off;
@@ -171,10 +197,10 @@ int resolve_max_context(const pa_pool* pool, int32_t max_blocks_per_seq, int32_t
   return (int)std::min<int64_t>(m, INT32_MAX);
 }
 
-template <typename T, int D>
+template <typename T, int D, int G>
 cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
-  using Cfg = DecodeKernelCfg<T, D>;
-  auto kernel = decode_kernel_ptr<T, D>();
+  using Cfg = DecodeKernelCfg<T, D, G>;
+  auto kernel = decode_kernel_ptr<T, D, G>();
   const size_t smem = Cfg::smem_bytes(a.partition_size);
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Cfg::THREADS, smem);
@@ -184,6 +210,16 @@ cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStrea
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
   kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_grouped(int G, const DecodeArgs& a, const DeviceState& dev, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode<T, D, 1>(a, dev, s);
+    case 2: return launch_decode<T, D, 2>(a, dev, s);
+    case 4: return launch_decode<T, D, 4>(a, dev, s);
+    default: return launch_decode<T, D, 8>(a, dev, s);
+  }
 }
 
 // One warp waits on a barrier that expects two arrivals but gets one.
@@ -220,6 +256,7 @@ pa_status pa_pool_create(int64_t num_blocks, int32_t block_size, int32_t heads, 
   p.heads = heads;
   p.head_dim = head_dim;
   p.dtype = dtype;
+  p.q_per_kv = 1;
   p.elem_bytes = dtype == PA_F32 ? 4 : 2;
   p.token_stride = head_dim;
   p.head_stride = (int64_t)block_size * head_dim;
@@ -228,6 +265,18 @@ pa_status pa_pool_create(int64_t num_blocks, int32_t block_size, int32_t heads, 
   pa_status st = check_pool(&p);
   if (st != PA_OK) return st;
   *out = p;
+  return PA_OK;
+}
+
+pa_status pa_pool_set_query_heads(pa_pool* pool, int32_t num_q_heads) {
+  if (!pool) return fail(PA_ERR_INVALID_ARG, "pa_pool_set_query_heads: pool is null");
+  if (num_q_heads <= 0 || num_q_heads % pool->heads != 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_pool_set_query_heads: query heads must be a positive multiple of KV heads");
+  const int32_t g = num_q_heads / pool->heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4 or 8");
+  pool->q_per_kv = g;
   return PA_OK;
 }
 
@@ -267,7 +316,9 @@ pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
   const int max_parts = std::max(1, (maxL + ps - 1) / ps);
-  *bytes = layout_for(num_seqs, pool->heads, max_parts, pool->head_dim).total;
+  *bytes = layout_for(num_seqs, (int64_t)pool->heads * pool->q_per_kv, max_parts, pool->head_dim,
+                      pool->q_per_kv)
+               .total;
   return PA_OK;
 }
 
@@ -289,13 +340,15 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
   if ((st = device_state(dev)) != PA_OK) return st;
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
-  const int head_groups = (pool->heads + kDecodeWarps - 1) / kDecodeWarps;
+  const int G = pool->q_per_kv;
+  const int head_groups = (pool->heads + rings_for(G) - 1) / rings_for(G);
   const int ps = partition_size != 0
                      ? partition_size
                      : auto_partition(num_seqs, head_groups, maxL,
                                       (*dev)->num_sms * (*dev)->decode_ctas_per_sm);
   const int max_parts = std::max(1, (maxL + ps - 1) / ps);
-  const WorkspaceLayout w = layout_for(num_seqs, pool->heads, max_parts, pool->head_dim);
+  const WorkspaceLayout w =
+      layout_for(num_seqs, (int64_t)pool->heads * G, max_parts, pool->head_dim, G);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(PA_ERR_WORKSPACE, "decode: workspace missing, not 256-byte aligned or too small");
   char* ws = static_cast<char*>(workspace);
@@ -312,7 +365,8 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   a->max_blocks_per_seq = max_blocks_per_seq;
   a->num_seqs = num_seqs;
   a->heads = pool->heads;
-  a->head_groups = (pool->heads + kDecodeWarps - 1) / kDecodeWarps;
+  a->q_per_kv = G;
+  a->head_groups = head_groups;
   a->partition_size = ps;
   a->max_parts = max_parts;
   a->max_context_len = maxL;
@@ -329,12 +383,14 @@ pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState
                      cudaStream_t s) {
   cudaError_t e;
   switch (pool->dtype * 1000 + pool->head_dim) {
-    case PA_F32 * 1000 + 64: e = launch_decode<float, 64>(a, dev, s); break;
-    case PA_F32 * 1000 + 128: e = launch_decode<float, 128>(a, dev, s); break;
-    case PA_F16 * 1000 + 64: e = launch_decode<__half, 64>(a, dev, s); break;
-    case PA_F16 * 1000 + 128: e = launch_decode<__half, 128>(a, dev, s); break;
-    case PA_BF16 * 1000 + 64: e = launch_decode<__nv_bfloat16, 64>(a, dev, s); break;
-    case PA_BF16 * 1000 + 128: e = launch_decode<__nv_bfloat16, 128>(a, dev, s); break;
+    case PA_F32 * 1000 + 64: e = launch_grouped<float, 64>(pool->q_per_kv, a, dev, s); break;
+    case PA_F32 * 1000 + 128: e = launch_grouped<float, 128>(pool->q_per_kv, a, dev, s); break;
+    case PA_F16 * 1000 + 64: e = launch_grouped<__half, 64>(pool->q_per_kv, a, dev, s); break;
+    case PA_F16 * 1000 + 128: e = launch_grouped<__half, 128>(pool->q_per_kv, a, dev, s); break;
+    case PA_BF16 * 1000 + 64: e = launch_grouped<__nv_bfloat16, 64>(pool->q_per_kv, a, dev, s); break;
+    case PA_BF16 * 1000 + 128:
+      e = launch_grouped<__nv_bfloat16, 128>(pool->q_per_kv, a, dev, s);
+      break;
     default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
   }
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode launch");

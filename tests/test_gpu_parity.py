@@ -361,3 +361,71 @@ def test_fused_append_planned_over_layers():
         want, wk, wv = oracle_append_and_decode(layer_case)
         assert np.array_equal(bits(kp), bits(wk)) and np.array_equal(bits(vp), bits(wv))
         assert_parity(out, want, f"fused planned layer {layer}")
+
+
+# ---- grouped-query attention ------------------------------------------------------------
+
+@pytest.mark.parametrize("group", [2, 4, 8])
+@pytest.mark.parametrize("dtype,head_dim", [(np.float16, 128), (np.float32, 64)])
+def test_gqa_matches_oracle_and_replicated_mha(group, dtype, head_dim):
+    """Query head h reads KV head h // group.  The result must match the
+    oracle and be bit-identical to MHA over a pool whose KV heads are
+    repeated group times (same arithmetic per query head)."""
+    kv_heads = 3
+    lens = [1, 15, 16, 17, 300, 513, 1024, 2048, 0]
+    case = syn.decode_case(41, lens, kv_heads, head_dim, dtype, max_blocks=130)
+    rng = np.random.default_rng(42)
+    qg = rng.standard_normal((len(lens), kv_heads * group, head_dim)).astype(dtype)
+    NB = case["k_pool"].shape[0]
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    kp, vp = dev(case["k_pool"]), dev(case["v_pool"])
+    pool = pa.pa_pool_create(NB, 16, kv_heads, head_dim, TORCH[dtype])
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    out = torch.empty((len(lens), kv_heads * group, head_dim), dtype=TORCH[dtype], device="cuda")
+    ws = workspace_for(pool, len(lens), bt.shape[1])
+    q = dev(qg)
+    pa.pa_decode_attention(pool, q, kp, vp, bt, cl, case["scale"], out, ws)
+    assert pa.pa_device_errors() == 0
+    ref = oracle.decode_attention(qg, case["k_pool"], case["v_pool"], case["block_tables"],
+                                  case["context_lens"], case["scale"])
+    assert_parity(out, ref, f"gqa x{group}")
+    # MHA over repeated KV heads
+    kr = np.ascontiguousarray(np.repeat(case["k_pool"], group, axis=1))
+    vr = np.ascontiguousarray(np.repeat(case["v_pool"], group, axis=1))
+    pool_r = pa.pa_pool_create(NB, 16, kv_heads * group, head_dim, TORCH[dtype])
+    out_r = torch.empty_like(out)
+    ws_r = workspace_for(pool_r, len(lens), bt.shape[1])
+    pa.pa_decode_attention(pool_r, q, dev(kr), dev(vr), bt, cl, case["scale"], out_r, ws_r)
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(out, out_r)
+
+
+@pytest.mark.parametrize("group", [4, 8])
+def test_gqa_fused_append(group):
+    kv_heads = 2
+    lens = [3, 16, 17, 600, 1, 2048]
+    case = syn.decode_case(43, lens, kv_heads, 128, np.float16, max_blocks=130)
+    rng = np.random.default_rng(44)
+    qg = rng.standard_normal((len(lens), kv_heads * group, 128)).astype(np.float16)
+    NB = case["k_pool"].shape[0]
+    pool = pa.pa_pool_create(NB, 16, kv_heads, 128, torch.float16)
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    kp, vp = dev(case["k_pool"]), dev(case["v_pool"])
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    out = torch.empty((len(lens), kv_heads * group, 128), dtype=torch.float16, device="cuda")
+    ws = workspace_for(pool, len(lens), bt.shape[1])
+    pa.pa_decode_append_attention(pool, dev(qg), dev(case["k_new"]), dev(case["v_new"]), kp, vp,
+                                  bt, cl, case["scale"], out, ws)
+    assert pa.pa_device_errors() == 0
+    want_case = dict(case, q=qg)
+    kh, vh = case["k_pool"].copy(), case["v_pool"].copy()
+    slots = np.array([oracle.slot_of_c(case["block_tables"][s], int(L) - 1)
+                      for s, L in enumerate(lens)], dtype=np.int32)
+    oracle.reshape_and_cache(case["k_new"], case["v_new"], slots, kh, vh)
+    ref = oracle.decode_attention(qg, kh, vh, case["block_tables"], case["context_lens"],
+                                  case["scale"])
+    assert np.array_equal(bits(kp), bits(kh)) and np.array_equal(bits(vp), bits(vh))
+    assert_parity(out, ref, f"gqa fused x{group}")
+
+
+TORCH = {np.float16: torch.float16, np.float32: torch.float32}
