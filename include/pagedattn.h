@@ -209,6 +209,42 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
                                              int32_t partition_size, void* stream);
 
 /*
+ * Decode over shared prefixes ("Atención paginada en modelos de lenguaje
+ * grandes (LLM)", 7minutos.es, section 3: requests with the same system
+ * prompt point at the same physical pages; "PagedAttention" wiki mirror,
+ * "Descripció": blocks shared across requests and branches).  Same result as
+ * pa_decode_attention, computed so that each shared block is read once for
+ * all the sequences holding it.
+ * Groups (device int32 arrays, CSR): members of group g are
+ * group_members[group_offsets[g] .. group_offsets[g+1]); they all hold the
+ * same physical blocks as the group's first member in their first
+ * group_blocks[g] table entries, and those blocks are full (16 tokens).
+ * A tensor-core kernel attends every member's query heads to the shared
+ * blocks (one partial result per 16-block chunk); the decode kernel attends
+ * each sequence to the rest of its context and merges everything by
+ * log-sum-exp.  fp16/bf16 pools only (PA_ERR_UNSUPPORTED for fp32).
+ * max_group_size and max_shared_blocks bound the group sizes and
+ * group_blocks (launch sizing).  A member that is too short, holds
+ * different blocks or belongs to two groups raises PA_DEVERR_CONTEXT_LEN and
+ * attends to its whole context on its own, so the result stays correct.
+ * Workspace: pa_decode_shared_prefix_workspace_bytes (max_shared_blocks
+ * extra slots per head).  pa_find_shared_prefixes builds groups from host
+ * block tables.
+ */
+pa_status pa_decode_shared_prefix_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
+                                                  int32_t max_blocks_per_seq,
+                                                  int32_t max_context_len, int32_t partition_size,
+                                                  int32_t max_shared_blocks, size_t* bytes);
+
+pa_status pa_decode_attention_shared_prefix(
+    const pa_pool* pool, const void* q, const void* k_pool, const void* v_pool,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+    int32_t num_seqs, const int32_t* group_offsets, const int32_t* group_members,
+    const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
+    int32_t max_shared_blocks, int32_t max_context_len, float scale, void* out, void* workspace,
+    size_t workspace_bytes, int32_t partition_size, void* stream);
+
+/*
  * Decode attention that allocates nothing.  Same computation, arguments and
  * errors as pa_decode_attention, minus the workspace: the plan and split-K
  * partials live in a static device buffer inside the library of
@@ -310,6 +346,22 @@ pa_status pa_fork_table(pa_allocator* a, const int32_t* src_table, int32_t num_b
 
 /* Drop the sequence's reference to each of its blocks (request finished). */
 pa_status pa_release_table(pa_allocator* a, const int32_t* block_table, int32_t num_blocks);
+
+/*
+ * Host helper: find shared prefixes in host block tables.  Sequences whose
+ * first table entries name the same block are candidates; a candidate set of
+ * two or more becomes a group whose shared length is the longest run of
+ * leading full blocks every member has in common (at least
+ * min_shared_blocks, else no group).  Outputs (host arrays sized num_seqs + 1,
+ * num_seqs, num_seqs): CSR offsets, members in table order, shared blocks;
+ * *num_groups, *max_group_size, *max_shared_blocks.
+ */
+pa_status pa_find_shared_prefixes(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t block_size, int32_t min_shared_blocks,
+                                  int32_t* group_offsets, int32_t* group_members,
+                                  int32_t* group_blocks, int32_t* num_groups,
+                                  int32_t* max_group_size, int32_t* max_shared_blocks);
 
 /* Host helper for tables built elsewhere: slot of the last token of each
  * sequence, block_tables[s][(L-1)/bs] * bs + (L-1) % bs, or -1 when L == 0.

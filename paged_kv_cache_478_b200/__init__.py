@@ -82,6 +82,12 @@ def lib():
                                                    i32, ctypes.c_float, vp, vp, sz, i32, vp],
             "pa_decode_attention_static": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, i32,
                                            ctypes.c_float, vp, i32, vp],
+            "pa_decode_shared_prefix_workspace_bytes": [P(pa_pool), i32, i32, i32, i32, i32, P(sz)],
+            "pa_decode_attention_shared_prefix": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, vp, vp,
+                                                  vp, i32, i32, i32, i32, ctypes.c_float, vp, vp,
+                                                  sz, i32, vp],
+            "pa_find_shared_prefixes": [vp, i32, vp, i32, i32, i32, vp, vp, vp, P(i32), P(i32),
+                                        P(i32)],
             "pa_copy_blocks": [P(pa_pool), vp, vp, vp, i32, vp],
             "pa_device_errors": [vp, P(ctypes.c_uint32)],
             "pa_selftest_wait_timeout": [vp],
@@ -296,6 +302,62 @@ def pa_decode_append_attention_planned(pool, q, k_new, v_new, k_pool, v_pool, bl
         _check_pool_tensor(pool, v_pool, "v_pool"),
         _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], S,
         max_context_len, float(scale), _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
+
+
+def pa_find_shared_prefixes(block_tables, context_lens, min_shared_blocks=1, block_size=16):
+    """Host helper: shared-prefix groups from host block tables.  Returns a
+    dict of numpy arrays (offsets, members, blocks) and the launch bounds."""
+    import numpy as np
+
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = cl.shape[0]
+    offs = np.zeros(S + 1, dtype=np.int32)
+    mem = np.zeros(max(S, 1), dtype=np.int32)
+    blk = np.zeros(max(S, 1), dtype=np.int32)
+    ng, mg, mb = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().pa_find_shared_prefixes(bt.ctypes.data, bt.shape[1], cl.ctypes.data, S, block_size,
+                                         min_shared_blocks, offs.ctypes.data, mem.ctypes.data,
+                                         blk.ctypes.data, ctypes.byref(ng), ctypes.byref(mg),
+                                         ctypes.byref(mb)))
+    n = ng.value
+    return dict(offsets=offs[:n + 1].copy(), members=mem[:offs[n]].copy(), blocks=blk[:n].copy(),
+                num_groups=n, max_group_size=mg.value, max_shared_blocks=mb.value)
+
+
+def pa_decode_shared_prefix_workspace_bytes(pool, num_seqs, max_blocks_per_seq, max_shared_blocks,
+                                            max_context_len=0, partition_size=0) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().pa_decode_shared_prefix_workspace_bytes(
+        ctypes.byref(pool), num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+        max_shared_blocks, ctypes.byref(n)))
+    return n.value
+
+
+def pa_decode_attention_shared_prefix(pool, q, k_pool, v_pool, block_tables, context_lens, groups,
+                                      scale, out, workspace, max_context_len=0, partition_size=0,
+                                      stream=None):
+    """groups: dict with device int32 tensors offsets, members, blocks and
+    ints num_groups, max_group_size, max_shared_blocks (see
+    pa_find_shared_prefixes for the host-side arrays)."""
+    torch = _torch()
+    S = q.shape[0]
+    if tuple(q.shape) != (S, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [num_seqs, query heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks], context_lens [num_seqs]")
+    dt = _pool_torch_dtype(pool)
+    ng = groups["num_groups"]
+    gp = [_dev_ptr(groups[k], k, torch.int32) if ng > 0 else None
+          for k in ("offsets", "members", "blocks")]
+    _check(lib().pa_decode_attention_shared_prefix(
+        ctypes.byref(pool), _dev_ptr(q, "q", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
+        _check_pool_tensor(pool, v_pool, "v_pool"),
+        _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev_ptr(context_lens, "context_lens", torch.int32), S, gp[0], gp[1], gp[2], ng,
+        groups["max_group_size"], groups["max_shared_blocks"], max_context_len, float(scale),
+        _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
 
 

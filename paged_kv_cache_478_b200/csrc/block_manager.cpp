@@ -15,6 +15,7 @@
 #include <functional>
 #include <new>
 #include <queue>
+#include <unordered_map>
 #include <vector>
 
 #include "pagedattn.h"
@@ -163,6 +164,62 @@ pa_status pa_release_table(pa_allocator* a, const int32_t* block_table, int32_t 
     if (!live(a, block_table[i]))
       return pa::fail(PA_ERR_INVALID_ARG, "pa_release_table: block not allocated");
   for (int32_t i = 0; i < num_blocks; ++i) pa_free_block(a, block_table[i]);
+  return PA_OK;
+}
+
+pa_status pa_find_shared_prefixes(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t block_size, int32_t min_shared_blocks,
+                                  int32_t* group_offsets, int32_t* group_members,
+                                  int32_t* group_blocks, int32_t* num_groups,
+                                  int32_t* max_group_size, int32_t* max_shared_blocks) {
+  if (num_seqs < 0 || block_size <= 0 || max_blocks_per_seq <= 0 || min_shared_blocks < 1)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_find_shared_prefixes: bad size");
+  if (!group_offsets || !num_groups || !max_group_size || !max_shared_blocks ||
+      (num_seqs > 0 && (!block_tables || !context_lens || !group_members || !group_blocks)))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_find_shared_prefixes: null argument");
+  auto row = [&](int32_t s) { return block_tables + static_cast<int64_t>(s) * max_blocks_per_seq; };
+  auto full_blocks = [&](int32_t s) {
+    return std::min<int64_t>(max_blocks_per_seq, std::max(0, context_lens[s]) / block_size);
+  };
+  // candidates keyed by their first block, in order of first appearance
+  std::unordered_map<int32_t, size_t> slot_of_key;
+  std::vector<std::vector<int32_t>> cand;
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    if (full_blocks(s) < min_shared_blocks) continue;
+    const int32_t key = row(s)[0];
+    auto it = slot_of_key.find(key);
+    if (it == slot_of_key.end()) {
+      slot_of_key.emplace(key, cand.size());
+      cand.push_back({s});
+    } else {
+      cand[it->second].push_back(s);
+    }
+  }
+  int32_t ng = 0, members = 0, max_size = 0, max_blocks = 0;
+  group_offsets[0] = 0;
+  for (const auto& c : cand) {
+    if (c.size() < 2) continue;
+    int64_t lcp = full_blocks(c[0]);
+    const int32_t* r0 = row(c[0]);
+    for (size_t i = 1; i < c.size(); ++i) {
+      const int32_t* r = row(c[i]);
+      const int64_t lim = std::min<int64_t>(lcp, full_blocks(c[i]));
+      int64_t k = 0;
+      while (k < lim && r[k] == r0[k]) ++k;
+      lcp = k;
+    }
+    if (lcp < min_shared_blocks) continue;
+    for (int32_t s : c) group_members[members++] = s;
+    group_blocks[ng] = static_cast<int32_t>(lcp);
+    group_offsets[ng + 1] = members;
+    max_size = std::max<int32_t>(max_size, static_cast<int32_t>(c.size()));
+    max_blocks = std::max<int32_t>(max_blocks, static_cast<int32_t>(lcp));
+    ++ng;
+  }
+  *num_groups = ng;
+  *max_group_size = max_size;
+  *max_shared_blocks = max_blocks;
   return PA_OK;
 }
 

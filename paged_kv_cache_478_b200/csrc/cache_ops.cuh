@@ -12,52 +12,53 @@
 
 namespace pa {
 
-// One CTA per new token.  row_chunks = head_dim * elem_bytes / 16.
-// k_new/v_new: [T][H][row_chunks] chunks; pools: [NB][H][16][row_chunks].
-__global__ void __launch_bounds__(128)
+// One thread per 16-byte chunk of every new row (K and V), grid-stride, so a
+// small batch of tokens still puts enough copies in flight.
+// row_chunks = head_dim * elem_bytes / 16.  k_new/v_new: [T][H][row_chunks]
+// chunks; pools: [NB][H][16][row_chunks].
+__global__ void __launch_bounds__(256)
     reshape_and_cache_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                              const int32_t* __restrict__ slot_mapping, uint4* __restrict__ k_pool,
                              uint4* __restrict__ v_pool, int heads, int row_chunks,
-                             int64_t num_slots, uint32_t* err) {
-  const int t = blockIdx.x;
-  const int32_t slot = slot_mapping[t];
-  if (slot < 0) return;  // padding token
-  if (slot >= num_slots) {
-    if (threadIdx.x == 0) atomicOr(err, PA_DEVERR_SLOT);
-    return;
-  }
-  const int64_t blk = slot / 16, off = slot % 16;
-  const int n = heads * row_chunks;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int h = i / row_chunks, c = i % row_chunks;
+                             int64_t num_tokens, int64_t num_slots, uint32_t* err) {
+  const int64_t per_token = (int64_t)heads * row_chunks;
+  const int64_t total = num_tokens * per_token;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t rem = i - t * per_token;
+    const int32_t slot = slot_mapping[t];
+    if (slot < 0) continue;  // padding token
+    if (slot >= num_slots) {
+      if (rem == 0) atomicOr(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t h = rem / row_chunks, c = rem - h * row_chunks;
+    const int64_t blk = slot / 16, off = slot % 16;
     const int64_t dst = ((blk * heads + h) * 16 + off) * row_chunks + c;
-    const int64_t src = (int64_t)t * n + i;
-    k_pool[dst] = k_new[src];
-    v_pool[dst] = v_new[src];
+    k_pool[dst] = k_new[i];
+    v_pool[dst] = v_new[i];
   }
 }
 
-// grid (num_pairs, split): CTA y of pair x copies its 1/split share of the
-// block (block_chunks 16-byte chunks) for K and for V.
+// One thread per 16-byte chunk of every (src, dst) block pair, grid-stride.
+// block_chunks = heads * 16 * head_dim * elem_bytes / 16.
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
-                       const int32_t* __restrict__ pairs, int64_t num_blocks,
+                       const int32_t* __restrict__ pairs, int64_t num_pairs, int64_t num_blocks,
                        int64_t block_chunks, uint32_t* err) {
-  const int32_t src = pairs[2 * blockIdx.x], dst = pairs[2 * blockIdx.x + 1];
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, PA_DEVERR_PAIR);
-    return;
-  }
-  const int64_t per = (block_chunks + gridDim.y - 1) / gridDim.y;
-  const int64_t lo = blockIdx.y * per;
-  const int64_t hi = min(block_chunks, lo + per);
-  const uint4* ks = k_pool + (int64_t)src * block_chunks;
-  const uint4* vs = v_pool + (int64_t)src * block_chunks;
-  uint4* kd = k_pool + (int64_t)dst * block_chunks;
-  uint4* vd = v_pool + (int64_t)dst * block_chunks;
-  for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) {
-    kd[i] = ks[i];
-    vd[i] = vs[i];
+  const int64_t total = num_pairs * block_chunks;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t pr = i / block_chunks;
+    const int64_t c = i - pr * block_chunks;
+    const int32_t src = pairs[2 * pr], dst = pairs[2 * pr + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (c == 0) atomicOr(err, PA_DEVERR_PAIR);
+      continue;
+    }
+    k_pool[(int64_t)dst * block_chunks + c] = k_pool[(int64_t)src * block_chunks + c];
+    v_pool[(int64_t)dst * block_chunks + c] = v_pool[(int64_t)src * block_chunks + c];
   }
 }
 

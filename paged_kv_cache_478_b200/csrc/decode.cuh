@@ -64,7 +64,17 @@ struct DecodeArgs {
   void* out;
   PlanHeader* plan;
   int32_t* lens;    // [S] clamped context lengths
-  int32_t* nparts;  // [S] partitions per sequence (>= 1)
+  int32_t* nparts;  // [S] partial results per sequence (>= 1): own partitions + shared chunks
+  int32_t* nitems;  // [S] own partitions (work items whose arrival triggers the merge)
+  int32_t* base;    // [S] first token of the sequence's own part (after its shared prefix)
+  int32_t* shared_of;  // [S] shared-prefix group of the sequence, or -1
+  // shared-prefix groups (null when there are none): CSR members, shared leading blocks
+  const int32_t* group_offsets;
+  const int32_t* group_members;
+  const int32_t* group_blocks;
+  int32_t num_groups;
+  int32_t max_shared_blocks;
+  int32_t shared_chunk;  // shared blocks per partial result
   int2* pairs;      // [S * max_parts] work pairs (s, p)
   float2* part_ml;  // [S][H][max_parts] (running max in log2 units, sum of weights)
   float* part_acc;  // [S][H][max_parts][D] unnormalised partial outputs
@@ -87,13 +97,12 @@ struct DecodeArgs {
 // ---- plan: one CTA orders the work ------------------------------------------------
 
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
-  extern __shared__ int32_t bucket[];  // [nb + 1]: index 0 = empty sequences
+  extern __shared__ int32_t bucket[];  // [nb + 1]: index 0 = sequences with no own tokens
   __shared__ int32_t n_full;
   const int PS = a.partition_size;
   const int nb = PS / kBlock;
   for (int i = threadIdx.x; i <= nb; i += blockDim.x) bucket[i] = 0;
   if (threadIdx.x == 0) n_full = 0;
-  __syncthreads();
   const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     int L = a.context_lens[s];
@@ -102,19 +111,69 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
       L = L < 0 ? 0 : cap;
     }
     a.lens[s] = L;
+    a.shared_of[s] = -1;
     for (int g = 0; g < a.head_groups; ++g) a.merge_cnt[(int64_t)s * a.head_groups + g] = 0;
-    const int full = L / PS, rem = L % PS;
-    a.nparts[s] = max(1, full + (rem > 0 ? 1 : 0));
+  }
+  __syncthreads();
+  // shared-prefix groups: a member joins if its table starts with the first
+  // member's blocks and it is long enough; anything else is reported and the
+  // sequence attends to its whole context on its own
+  if (a.group_offsets != nullptr) {
+    // groups in turn, their members spread over the CTA's threads
+    for (int g = 0; g < a.num_groups; ++g) {
+      const int m0 = a.group_offsets[g], m1 = a.group_offsets[g + 1];
+      const int nbk = a.group_blocks[g];
+      if (m1 <= m0 || nbk <= 0) continue;
+      if (nbk > a.max_shared_blocks || nbk > a.max_blocks_per_seq || m0 < 0) {
+        if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+        continue;
+      }
+      const int rep = a.group_members[m0];
+      if (rep < 0 || rep >= a.num_seqs || a.lens[rep] < nbk * kBlock) {
+        if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+        continue;
+      }
+      const int32_t* rt = a.block_tables + (int64_t)rep * a.max_blocks_per_seq;
+      for (int m = m0 + threadIdx.x; m < m1; m += blockDim.x) {
+        const int s = a.group_members[m];
+        bool ok = s >= 0 && s < a.num_seqs && a.lens[s] >= nbk * kBlock;
+        if (ok) {
+          const int32_t* t = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+          int diff = 0;  // independent loads, no early exit, so they overlap
+#pragma unroll 8
+          for (int j = 0; j < nbk; ++j) diff |= t[j] ^ rt[j];
+          ok = diff == 0;
+        }
+        if (!ok) {
+          atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+        } else if (atomicCAS(&a.shared_of[s], -1, g) != -1) {
+          atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+    const int L = a.lens[s];
+    const int g = a.shared_of[s];
+    const int sb = g >= 0 ? a.group_blocks[g] : 0;
+    const int base = sb * kBlock;
+    const int U = L - base;  // the sequence's own tokens
+    const int full = U / PS, rem = U % PS;
+    const int ni = max(1, full + (rem > 0 ? 1 : 0));
+    a.base[s] = base;
+    a.nitems[s] = ni;
+    a.nparts[s] = ni + (sb > 0 ? (sb + a.shared_chunk - 1) / a.shared_chunk : 0);
     if (full > 0) {
       const int pos = atomicAdd(&n_full, full);
       for (int p = 0; p < full; ++p) a.pairs[pos + p] = make_int2(s, p);
     }
-    if (L == 0 || rem > 0) atomicAdd(&bucket[L == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
+    if (U == 0 || rem > 0) atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = n_full;
-    for (int b = nb; b >= 0; --b) {  // biggest remainders first, empty sequences last
+    for (int b = nb; b >= 0; --b) {  // biggest remainders first, empty ones last
       const int c = bucket[b];
       bucket[b] = run;
       run += c;
@@ -126,11 +185,11 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
   }
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
-    const int L = a.lens[s];
-    const int rem = L % PS;
-    if (L == 0 || rem > 0) {
-      const int pos = atomicAdd(&bucket[L == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
-      a.pairs[pos] = make_int2(s, L / PS);
+    const int U = a.lens[s] - a.base[s];
+    const int rem = U % PS;
+    if (U == 0 || rem > 0) {
+      const int pos = atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
+      a.pairs[pos] = make_int2(s, U / PS);
     }
   }
 }
@@ -301,13 +360,14 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
     const int s = pr.x, p = pr.y;
     const int L = a.lens[s];
     const int np = a.nparts[s];
+    const int ni = a.nitems[s];
     const bool split = np > 1;
-    const int tok0 = p * PS;
+    const int tok0 = a.base[s] + p * PS;
     const int ntok = max(0, min(L, tok0 + PS) - tok0);
     const int nblk = (ntok + kBlock - 1) / kBlock;
     const int blk0 = tok0 / kBlock;
     // the item holding the sequence's last token appends the new one (fused mode)
-    const bool append = a.k_new != nullptr && L > 0 && p == np - 1;
+    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1;
     const int new_row = (L - 1) % kBlock;  // in-block offset of the appended token
 
     // block-table slice of this partition, bounds-checked once
@@ -474,9 +534,9 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
       if (threadIdx.x == 0) {
         int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
         __threadfence();
-        const int arrived = atomicAdd(cnt, 1) + 1;
-        s_merge = arrived == np && !s_abort;
-        if (arrived == np) *cnt = 0;  // re-arm for the next launch on this plan
+        const int arrived = atomicAdd(cnt, 1) + 1;  // shared-prefix partials are already written
+        s_merge = arrived == ni && !s_abort;
+        if (arrived == ni) *cnt = 0;  // re-arm for the next launch on this plan
       }
       __syncthreads();
       if (s_merge && kvh < HK) {

@@ -10,6 +10,7 @@
 
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "shared_prefix.cuh"
 #include "pagedattn.h"
 #include "status.h"
 
@@ -146,9 +147,16 @@ pa_status check_pool(const pa_pool* pool) {
 }
 
 struct WorkspaceLayout {
-  size_t header = 0, lens = 0, nparts = 0, merge_cnt = 0, pairs = 0, part_ml = 0, part_acc = 0,
-         total = 0;
+  size_t header = 0, lens = 0, nparts = 0, nitems = 0, base = 0, shared_of = 0, merge_cnt = 0,
+         pairs = 0, part_ml = 0, part_acc = 0, total = 0;
 };
+
+constexpr int kSharedChunk = 16;  // shared-prefix blocks per partial result
+
+// Partial-result slots per (sequence, head): own partitions + shared chunks.
+int total_parts(int maxL, int ps, int max_shared_blocks) {
+  return std::max(1, (maxL + ps - 1) / ps) + (max_shared_blocks + kSharedChunk - 1) / kSharedChunk;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -161,6 +169,12 @@ WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D, i
   w.lens = off;
   off = align256(off + S * 4);
   w.nparts = off;
+  off = align256(off + S * 4);
+  w.nitems = off;
+  off = align256(off + S * 4);
+  w.base = off;
+  off = align256(off + S * 4);
+  w.shared_of = off;
   off = align256(off + S * 4);
   w.merge_cnt = off;
   off = align256(off + S * ((H / G + rings_for(G) - 1) / rings_for(G)) * 4);
@@ -294,32 +308,41 @@ pa_status pa_reshape_and_cache(const pa_pool* pool, const void* k_new, const voi
   DeviceState* dev;
   if ((st = device_state(&dev)) != PA_OK) return st;
   const int row_chunks = pool->head_dim * pool->elem_bytes / 16;
-  reshape_and_cache_kernel<<<num_tokens, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+  const int64_t total = (int64_t)num_tokens * pool->heads * row_chunks;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)dev->num_sms * 16);
+  reshape_and_cache_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping,
       static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pool->heads, row_chunks,
-      pool->num_blocks * pool->block_size, dev->err);
+      num_tokens, pool->num_blocks * pool->block_size, dev->err);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "reshape_and_cache launch");
 }
 
-pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
-                                    int32_t max_blocks_per_seq, int32_t max_context_len,
-                                    int32_t partition_size, size_t* bytes) {
+pa_status pa_decode_shared_prefix_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
+                                                  int32_t max_blocks_per_seq,
+                                                  int32_t max_context_len, int32_t partition_size,
+                                                  int32_t max_shared_blocks, size_t* bytes) {
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
-  if (!bytes) return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bytes is null");
-  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
-    return fail(PA_ERR_INVALID_ARG, "pa_decode_workspace_bytes: bad size");
+  if (!bytes) return fail(PA_ERR_INVALID_ARG, "workspace bytes: bytes is null");
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || max_shared_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace bytes: bad size");
   // partition_size 0: the automatic choice is never below kMinAutoPartition
   const int ps = partition_size == 0 ? kMinAutoPartition : partition_size;
   if (ps < kBlock || ps % kBlock != 0 || ps > kMaxPartition)
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
-  const int max_parts = std::max(1, (maxL + ps - 1) / ps);
-  *bytes = layout_for(num_seqs, (int64_t)pool->heads * pool->q_per_kv, max_parts, pool->head_dim,
-                      pool->q_per_kv)
+  *bytes = layout_for(num_seqs, (int64_t)pool->heads * pool->q_per_kv,
+                      total_parts(maxL, ps, max_shared_blocks), pool->head_dim, pool->q_per_kv)
                .total;
   return PA_OK;
+}
+
+pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
+                                    int32_t max_blocks_per_seq, int32_t max_context_len,
+                                    int32_t partition_size, size_t* bytes) {
+  return pa_decode_shared_prefix_workspace_bytes(pool, num_seqs, max_blocks_per_seq,
+                                                 max_context_len, partition_size, 0, bytes);
 }
 
 }  // extern "C"
@@ -330,7 +353,8 @@ namespace {
 // workspace pointers of a.
 pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_blocks_per_seq,
                          int32_t max_context_len, int32_t partition_size, void* workspace,
-                         size_t workspace_bytes, DecodeArgs* a, DeviceState** dev) {
+                         size_t workspace_bytes, DecodeArgs* a, DeviceState** dev,
+                         int32_t max_shared_blocks = 0) {
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
@@ -346,7 +370,7 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
                      ? partition_size
                      : auto_partition(num_seqs, head_groups, maxL,
                                       (*dev)->num_sms * (*dev)->decode_ctas_per_sm);
-  const int max_parts = std::max(1, (maxL + ps - 1) / ps);
+  const int max_parts = total_parts(maxL, ps, max_shared_blocks);
   const WorkspaceLayout w =
       layout_for(num_seqs, (int64_t)pool->heads * G, max_parts, pool->head_dim, G);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -356,6 +380,11 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   a->plan = reinterpret_cast<PlanHeader*>(ws + w.header);
   a->lens = reinterpret_cast<int32_t*>(ws + w.lens);
   a->nparts = reinterpret_cast<int32_t*>(ws + w.nparts);
+  a->nitems = reinterpret_cast<int32_t*>(ws + w.nitems);
+  a->base = reinterpret_cast<int32_t*>(ws + w.base);
+  a->shared_of = reinterpret_cast<int32_t*>(ws + w.shared_of);
+  a->max_shared_blocks = max_shared_blocks;
+  a->shared_chunk = kSharedChunk;
   a->pairs = reinterpret_cast<int2*>(ws + w.pairs);
   a->part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
   a->part_acc = reinterpret_cast<float*>(ws + w.part_acc);
@@ -520,6 +549,73 @@ pa_status pa_decode_append_attention(const pa_pool* pool, const void* q, const v
                                             stream);
 }
 
+pa_status pa_decode_attention_shared_prefix(
+    const pa_pool* pool, const void* q, const void* k_pool, const void* v_pool,
+    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+    int32_t num_seqs, const int32_t* group_offsets, const int32_t* group_members,
+    const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
+    int32_t max_shared_blocks, int32_t max_context_len, float scale, void* out, void* workspace,
+    size_t workspace_bytes, int32_t partition_size, void* stream) {
+  if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "shared prefix: negative size");
+  if (num_seqs == 0) return check_pool(pool);
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (pool->dtype == PA_F32)
+    return fail(PA_ERR_UNSUPPORTED, "shared prefix: fp16 or bf16 pools only (tensor-core path)");
+  st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
+  if (st != PA_OK) return st;
+  if (!context_lens) return fail(PA_ERR_INVALID_ARG, "shared prefix: context_lens is null");
+  if (num_groups > 0 && (!group_offsets || !group_members || !group_blocks))
+    return fail(PA_ERR_INVALID_ARG, "shared prefix: group arrays are null");
+  DecodeArgs a;
+  DeviceState* dev;
+  st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+                      workspace, workspace_bytes, &a, &dev, max_shared_blocks);
+  if (st != PA_OK) return st;
+  a.context_lens = context_lens;
+  if (num_groups > 0 && max_shared_blocks > 0 && max_group_size > 0) {
+    a.group_offsets = group_offsets;
+    a.group_members = group_members;
+    a.group_blocks = group_blocks;
+    a.num_groups = num_groups;
+  }
+  set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = launch_plan(a, s)) != PA_OK) return st;
+  if (a.group_offsets != nullptr) {
+    SharedPrefixArgs sp;
+    sp.group_offsets = group_offsets;
+    sp.group_members = group_members;
+    sp.group_blocks = group_blocks;
+    sp.num_groups = num_groups;
+    const int rows = max_group_size * pool->q_per_kv;
+    sp.row_tiles = (rows + 63) / 64;
+    sp.chunk_blocks = kSharedChunk;
+    const dim3 grid((unsigned)((int64_t)num_groups * sp.row_tiles), (unsigned)pool->heads,
+                    (unsigned)((max_shared_blocks + kSharedChunk - 1) / kSharedChunk));
+    if ((int64_t)num_groups * sp.row_tiles > INT32_MAX || grid.z > 65535 || grid.y > 65535)
+      return fail(PA_ERR_INVALID_ARG, "shared prefix: too many groups or blocks");
+    const bool bf16 = pool->dtype == PA_BF16;
+    if (pool->head_dim == 128) {
+      if (bf16)
+        shared_prefix_kernel<__nv_bfloat16, 128>
+            <<<grid, 128, SharedPrefixConfig<128>::smem_bytes(), s>>>(sp, a);
+      else
+        shared_prefix_kernel<__half, 128><<<grid, 128, SharedPrefixConfig<128>::smem_bytes(), s>>>(sp, a);
+    } else {
+      if (bf16)
+        shared_prefix_kernel<__nv_bfloat16, 64>
+            <<<grid, 128, SharedPrefixConfig<64>::smem_bytes(), s>>>(sp, a);
+      else
+        shared_prefix_kernel<__half, 64><<<grid, 128, SharedPrefixConfig<64>::smem_bytes(), s>>>(sp, a);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "shared prefix launch");
+  }
+  return launch_run(pool, a, *dev, s);
+}
+
 pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,
                          int32_t num_pairs, void* stream) {
   pa_status st = check_pool(pool);
@@ -532,10 +628,11 @@ pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const 
   DeviceState* dev;
   if ((st = device_state(&dev)) != PA_OK) return st;
   const int64_t block_chunks = pool->block_stride * pool->elem_bytes / 16;
-  const int split = (int)std::min<int64_t>(16, std::max<int64_t>(1, block_chunks / 1024));
-  copy_blocks_kernel<<<dim3(num_pairs, split), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, pool->num_blocks,
-      block_chunks, dev->err);
+  const int64_t total = (int64_t)num_pairs * block_chunks;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)dev->num_sms * 16);
+  copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs, num_pairs,
+      pool->num_blocks, block_chunks, dev->err);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks launch");
 }

@@ -142,3 +142,50 @@ def test_decode_slots_matches_the_oracle():
     assert got.tolist() == want
     lens[4] = 0
     assert pa.pa_decode_slots(tables, lens)[4] == -1
+
+
+def _prefix_tables():
+    """128 sequences share a 1000-token prefix (63 blocks), then each adds a
+    suffix; the first divergent write copies block 62 for all but the last."""
+    rng = np.random.default_rng(5)
+    bm = pa.BlockManager(4096)
+    S, P = 128, 1000
+    tables = np.full((S, 95), -1, dtype=np.int32)
+    lens = np.zeros(S, dtype=np.int32)
+    lens[0], _, _ = bm.append_tokens(tables[0], 0, P)
+    for s in range(1, S):
+        bm.fork_table(tables[0], 63, tables[s])
+        lens[s] = P
+    for s in range(S):
+        lens[s], _, _ = bm.append_tokens(tables[s], int(lens[s]), int(rng.integers(1, 513)))
+    return tables, lens
+
+
+def test_find_shared_prefixes_on_a_forked_prompt():
+    tables, lens = _prefix_tables()
+    g = pa.pa_find_shared_prefixes(tables, lens)
+    assert g["num_groups"] == 1 and g["max_group_size"] == 128
+    assert g["blocks"].tolist() == [62]        # block 62 was copied on write by 127 holders
+    assert g["members"].tolist() == list(range(128))
+    assert g["offsets"].tolist() == [0, 128]
+
+
+def test_find_shared_prefixes_hand_cases():
+    t = np.full((6, 6), -1, dtype=np.int32)
+    t[0, :5] = [7, 8, 9, 10, 11]
+    t[1, :5] = [7, 8, 9, 20, 21]   # shares 3 blocks with 0
+    t[2, :4] = [30, 31, 32, 33]    # alone
+    t[3, :3] = [40, 41, 42]
+    t[4, :3] = [40, 41, 50]        # shares 2 with 3
+    t[5, :2] = [7, 8]              # shares 2 with 0 and 1, but only 1 full block
+    lens = np.array([80, 80, 64, 48, 48, 20], dtype=np.int32)
+    g = pa.pa_find_shared_prefixes(t, lens)
+    # 5 has one full block (20 tokens), so the {0, 1, 5} group shares 1 block
+    assert g["num_groups"] == 2
+    assert g["members"].tolist() == [0, 1, 5, 3, 4]
+    assert g["blocks"].tolist() == [1, 2]
+    g2 = pa.pa_find_shared_prefixes(t, lens, min_shared_blocks=2)
+    # 5 no longer qualifies (one full block), so 0 and 1 share 3 blocks
+    assert g2["members"].tolist() == [0, 1, 3, 4]
+    assert g2["blocks"].tolist() == [3, 2]
+    assert g2["max_group_size"] == 2 and g2["max_shared_blocks"] == 3

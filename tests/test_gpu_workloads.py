@@ -224,3 +224,87 @@ def test_full_decode_step_sampled():
             checked += 1
         del kp, vp
     assert checked == len(sample_layers)
+
+
+def _groups_to_device(g):
+    d = dict(g)
+    for k in ("offsets", "members", "blocks"):
+        d[k] = dev(np.ascontiguousarray(g[k], dtype=np.int32))
+    return d
+
+
+def test_shared_prefix_path_on_the_forked_prompt():
+    """The tensor-core shared-prefix path on the 128-way shared system prompt:
+    the same answer as the oracle and as the plain decode path."""
+    case = syn.shared_prefix_case(seed=2)
+    S = 128
+    nb = 63 + S + sum(math.ceil(int(n) / BS) for n in case["suffix_lens"])
+    g = _gpu_shared_prefix(case, nb)
+    r = _oracle_shared_prefix(case, nb)
+    groups = pa.pa_find_shared_prefixes(g["tables"], g["lens"])
+    assert groups["num_groups"] == 1 and groups["blocks"].tolist() == [62]
+    pool = g["pool"]
+    q = dev(case["q"])
+    out = torch.empty_like(q)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(
+        pool, S, g["tables"].shape[1], groups["max_shared_blocks"]), dtype=torch.uint8,
+        device="cuda")
+    pa.pa_decode_attention_shared_prefix(pool, q, g["kp"], g["vp"], dev(g["tables"]),
+                                         dev(g["lens"]), _groups_to_device(groups),
+                                         case["scale"], out, ws)
+    assert pa.pa_device_errors() == 0
+    assert_parity(out, r["out"], "shared-prefix path")
+    assert_parity(out, g["out"].double().cpu().numpy(), "shared-prefix vs plain path")
+
+
+@pytest.mark.parametrize("dtype,group", [("f16", 1), ("bf16", 4), ("f16", 8)])
+def test_shared_prefix_groups_with_gqa_and_a_bad_member(dtype, group):
+    rng = np.random.default_rng(60 + group)
+    H, D = 2, 128
+    HQ = H * group
+    # group A: sequences 0-4 share 20 blocks; group B: 5-7 share 3 blocks; 8-9 alone
+    lens = np.array([400, 333, 321, 700, 1024, 60, 49, 64, 17, 250], dtype=np.int32)
+    nb = 400
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((10, 64), -1, dtype=np.int32)
+    pos = 0
+    shared_a = perm[pos:pos + 20]; pos += 20
+    shared_b = perm[pos:pos + 3]; pos += 3
+    for s, L in enumerate(lens):
+        n = math.ceil(int(L) / 16)
+        pre = shared_a if s < 5 else (shared_b if s < 8 else np.zeros(0, np.int32))
+        tables[s, :len(pre)] = pre
+        tables[s, len(pre):n] = perm[pos:pos + n - len(pre)]
+        pos += n - len(pre)
+    groups = pa.pa_find_shared_prefixes(tables, lens)
+    assert groups["num_groups"] == 2
+    assert groups["blocks"].tolist() == [20, 3]
+    # plant a member that does not hold the group's blocks: it must be reported
+    # and still get the right answer on its own
+    groups["members"] = np.concatenate([groups["members"][:5], [9], groups["members"][5:]])
+    groups["offsets"] = np.array([0, 6, 9], dtype=np.int32)
+    groups["max_group_size"] = 6
+    shape = (nb, H, BS, D)
+    kh = rng.standard_normal(shape).astype(np.float32)
+    vh = rng.standard_normal(shape).astype(np.float32)
+    qh = rng.standard_normal((10, HQ, D)).astype(np.float32)
+    if dtype == "bf16":
+        tdt = torch.bfloat16
+        kt, vt, qt = (torch.from_numpy(x).to(tdt) for x in (kh, vh, qh))
+        kb, vb, qb = (x.view(torch.int16).numpy().view(np.uint16) for x in (kt, vt, qt))
+        ref = oracle.decode_attention(qb, kb, vb, tables, lens, 1 / math.sqrt(D), dtype=oracle.BF16)
+    else:
+        tdt = torch.float16
+        kt, vt, qt = (torch.from_numpy(x.astype(np.float16)) for x in (kh, vh, qh))
+        ref = oracle.decode_attention(qt.numpy(), kt.numpy(), vt.numpy(), tables, lens,
+                                      1 / math.sqrt(D))
+    pool = pa.pa_pool_create(nb, BS, H, D, tdt)
+    pa.pa_pool_set_query_heads(pool, HQ)
+    q = qt.cuda()
+    out = torch.empty_like(q)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(pool, 10, 64, 20),
+                     dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention_shared_prefix(pool, q, kt.cuda(), vt.cuda(), dev(tables), dev(lens),
+                                         _groups_to_device(groups), 1 / math.sqrt(D), out, ws)
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN  # the planted member
+    assert_parity(out, ref, f"shared prefix {dtype} G={group}")
