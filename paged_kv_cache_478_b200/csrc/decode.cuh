@@ -134,20 +134,23 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
         continue;
       }
       const int32_t* rt = a.block_tables + (int64_t)rep * a.max_blocks_per_seq;
-      for (int m = m0 + threadIdx.x; m < m1; m += blockDim.x) {
+      // one warp per member: its lanes compare 32 table entries at a time
+      const int lane = threadIdx.x & 31;
+      for (int m = m0 + (threadIdx.x >> 5); m < m1; m += blockDim.x >> 5) {
         const int s = a.group_members[m];
         bool ok = s >= 0 && s < a.num_seqs && a.lens[s] >= nbk * kBlock;
         if (ok) {
           const int32_t* t = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-          int diff = 0;  // independent loads, no early exit, so they overlap
-#pragma unroll 8
-          for (int j = 0; j < nbk; ++j) diff |= t[j] ^ rt[j];
-          ok = diff == 0;
+          int diff = 0;
+          for (int j = lane; j < nbk; j += 32) diff |= t[j] ^ rt[j];
+          ok = !__any_sync(kFullMask, diff != 0);
         }
-        if (!ok) {
-          atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-        } else if (atomicCAS(&a.shared_of[s], -1, g) != -1) {
-          atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
+        if (lane == 0) {
+          if (!ok) {
+            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+          } else if (atomicCAS(&a.shared_of[s], -1, g) != -1) {
+            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
+          }
         }
       }
     }

@@ -1,0 +1,312 @@
+// Grouped-query decode on tensor cores (fp16 / bf16 pools).
+//
+// With G query heads per KV head, each staged (block, KV head) tile serves G
+// queries: per 16-token block that is a [G x D] . [D x 16] score product and
+// a [G x 16] . [16 x D] value product, i.e. two m16n8k16 chains with the G
+// query heads as the rows.  One warp owns one KV head of the work item and
+// all of its query heads, so the CUDA-core cost per byte no longer grows
+// with G.  The softmax weights enter P.V as a high part plus its rounding
+// residual, so bf16 operands do not cost the result precision.  The pipeline
+// is the MHA kernel's: a per-warp NSTAGE ring fed by
+// 1-D bulk copies on mbarriers, items from the plan's queue, split-K partials
+// merged by the last CTA to finish a sequence, optional fused append.  Rows
+// land in shared memory padded to D*2+16 bytes (one bulk copy per token row,
+// issued by 16 lanes for K and 16 for V), so ldmatrix reads are free of bank
+// conflicts; rows past the end of a ragged block are zero-filled instead of
+// copied, so stale pool contents never reach the product.
+#pragma once
+
+#include <math.h>
+#include <stdint.h>
+
+#include "decode.cuh"
+#include "device_utils.cuh"
+#include "mma_utils.cuh"
+
+namespace pa {
+
+template <typename T, int D, int NSTAGE>
+struct GqaConfig {
+  static constexpr int WARPS = 4;            // KV heads per work item, one per warp
+  static constexpr int THREADS = WARPS * 32;
+  static constexpr int ROW_BYTES = D * 2;
+  static constexpr int PITCH = ROW_BYTES + 16;
+  static constexpr int TILE_BYTES = kBlock * PITCH;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
+  static size_t smem_bytes(int partition_size) {
+    return (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
+           (size_t)(partition_size / kBlock) * 4;
+  }
+};
+
+template <typename T, int D, int NSTAGE>
+__global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
+  using Cfg = GqaConfig<T, D, NSTAGE>;
+  constexpr int KSTEPS = D / 16;
+  constexpr int NT = D / 8;
+  constexpr int WARPS = Cfg::WARPS;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * NSTAGE * Cfg::STAGE_BYTES);
+  int32_t* tbl = reinterpret_cast<int32_t*>(bars + WARPS * NSTAGE);
+  __shared__ int32_t s_item;
+  __shared__ int32_t s_abort;
+  __shared__ int32_t s_merge;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = a.q_per_kv;  // query heads per KV head, <= 8
+  const int HK = a.heads, HQ = a.heads * G;
+  const int PS = a.partition_size;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    mbar_init_fence();
+    s_abort = 0;
+  }
+  int32_t next = 0;
+  if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
+  const int32_t num_items = a.plan->num_items;
+  __syncthreads();
+
+  uint32_t fills = 0;
+  uint8_t* my_stages = stages + warp * NSTAGE * Cfg::STAGE_BYTES;
+  uint64_t* my_bars = bars + warp * NSTAGE;
+  // the query row (head within the group) of each accumulator half: lane/4 and lane/4 + 8
+  const int qrow = lane >> 2;
+  const bool row_ok = qrow < G;  // rows 8..15 are never used (G <= 8)
+
+  for (;;) {
+    if (threadIdx.x == 0) {
+      s_item = next;
+      if (next < num_items) next = atomicAdd(&a.plan->work_counter, 1);
+    }
+    __syncthreads();
+    const int item = s_item;
+    if (item >= num_items || s_abort) break;
+
+    const int2 pr = a.pairs[item / a.head_groups];
+    const int g = item % a.head_groups;
+    const int s = pr.x, p = pr.y;
+    const int L = a.lens[s];
+    const int np = a.nparts[s];
+    const int ni = a.nitems[s];
+    const bool split = np > 1;
+    const int tok0 = a.base[s] + p * PS;
+    const int ntok = max(0, min(L, tok0 + PS) - tok0);
+    const int nblk = (ntok + kBlock - 1) / kBlock;
+    const int blk0 = tok0 / kBlock;
+    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1;
+    const int new_row = (L - 1) % kBlock;
+
+    for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
+      int32_t b = a.block_tables[(int64_t)s * a.max_blocks_per_seq + blk0 + i];
+      if (b < 0 || b >= a.num_blocks) {
+        atomicOr(a.err, PA_DEVERR_BLOCK_ID);
+        b = 0;
+      }
+      tbl[i] = b;
+    }
+    __syncthreads();
+
+    const int kvh = g * WARPS + warp;
+    if (kvh < HK) {
+      // Q fragments of this KV head's query heads (rows >= G are zero)
+      uint32_t qa[KSTEPS][4];
+      {
+        const T* q0 = static_cast<const T*>(a.q) + ((int64_t)s * HQ + kvh * G + qrow) * D;
+        const int kc = (lane & 3) * 2;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          qa[ks][0] = row_ok ? *reinterpret_cast<const uint32_t*>(q0 + ks * 16 + kc) : 0u;
+          qa[ks][1] = 0u;
+          qa[ks][2] = row_ok ? *reinterpret_cast<const uint32_t*>(q0 + ks * 16 + kc + 8) : 0u;
+          qa[ks][3] = 0u;
+        }
+      }
+      float m_run = -INFINITY, l_run = 0.f;
+      float o[NT][2];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
+
+      const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
+      const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
+      const int64_t block_bytes = (int64_t)HK * kBlock * Cfg::ROW_BYTES;
+      // fill stage k with block bi: lanes 0-15 take K rows, 16-31 V rows; rows
+      // past the valid count are zeroed rather than copied
+      auto issue = [&](uint32_t k, int bi) {
+        const int st = k % NSTAGE;
+        const uint32_t bar = smem_addr(&my_bars[st]);
+        uint8_t* dst = my_stages + st * Cfg::STAGE_BYTES;
+        const int valid = min(kBlock, ntok - bi * kBlock);
+        const int row = lane & 15;
+        const bool is_v = lane >= 16;
+        fence_proxy_async_shared();
+        if (lane == 0) mbar_arrive_expect_tx(bar, 2 * valid * Cfg::ROW_BYTES);
+        __syncwarp();
+        uint8_t* rdst = dst + (is_v ? Cfg::TILE_BYTES : 0) + row * Cfg::PITCH;
+        if (row < valid) {
+          const char* src = (is_v ? vbase : kbase) + (int64_t)tbl[bi] * block_bytes +
+                            (int64_t)row * Cfg::ROW_BYTES;
+          bulk_copy_g2s(smem_addr(rdst), src, Cfg::ROW_BYTES, bar);
+        } else {
+#pragma unroll
+          for (int c = 0; c < Cfg::ROW_BYTES / 16; ++c)
+            reinterpret_cast<uint4*>(rdst)[c] = make_uint4(0, 0, 0, 0);
+        }
+      };
+
+      const uint32_t k0 = fills;
+      for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
+      bool ok = true;
+      int i = 0;
+      for (; i < nblk; ++i) {
+        const uint32_t k = k0 + i;
+        const int st = k % NSTAGE;
+        const bool landed = mbar_wait_bounded(smem_addr(&my_bars[st]), (k / NSTAGE) & 1u);
+        if (!__all_sync(kFullMask, landed)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();  // the zero-filled rows of this stage are visible to every lane
+        uint8_t* ktile = my_stages + st * Cfg::STAGE_BYTES;
+        uint8_t* vtile = ktile + Cfg::TILE_BYTES;
+        const int valid = min(kBlock, ntok - i * kBlock);
+        if (append && i == nblk - 1) {
+          // fused reshape_and_cache of the KV head's new row
+          if (lane < Cfg::ROW_BYTES / 16) {
+            const int64_t skv = (int64_t)s * HK + kvh;
+            const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + skv * D)[lane];
+            const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + skv * D)[lane];
+            reinterpret_cast<uint4*>(ktile + new_row * Cfg::PITCH)[lane] = kn;
+            reinterpret_cast<uint4*>(vtile + new_row * Cfg::PITCH)[lane] = vn;
+            const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * Cfg::ROW_BYTES;
+            reinterpret_cast<uint4*>(const_cast<char*>(kbase) + row_off)[lane] = kn;
+            reinterpret_cast<uint4*>(const_cast<char*>(vbase) + row_off)[lane] = vn;
+          }
+          __syncwarp();
+        }
+
+        // S = Q K^T: sc[0] tokens 0-7, sc[1] tokens 8-15 (rows 0-7 in c0,c1)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+          const int row = (lane & 7) + ((lane >> 4) << 3);
+          const int col8 = ((lane >> 3) & 1) * 8;
+#pragma unroll
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            uint32_t b[4];
+            ldmatrix_x4(b, smem_addr(ktile + row * Cfg::PITCH + (ks * 16 + col8) * 2));
+            mma16816<T>(sc[0], qa[ks], b[0], b[1]);
+            mma16816<T>(sc[1], qa[ks], b[2], b[3]);
+          }
+        }
+        const int t0 = (lane & 3) * 2;  // token of c0 within each 8-token half
+        float x0 = t0 < valid ? sc[0][0] * a.scale_log2 : -INFINITY;
+        float x1 = t0 + 1 < valid ? sc[0][1] * a.scale_log2 : -INFINITY;
+        float x2 = t0 + 8 < valid ? sc[1][0] * a.scale_log2 : -INFINITY;
+        float x3 = t0 + 9 < valid ? sc[1][1] * a.scale_log2 : -INFINITY;
+        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = exp2f(m_run - m_new);
+        const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
+        const float p2 = exp2f(x2 - m_new), p3 = exp2f(x3 - m_new);
+        float sum = (p0 + p1) + (p2 + p3);
+        sum += __shfl_xor_sync(kFullMask, sum, 1);
+        sum += __shfl_xor_sync(kFullMask, sum, 2);
+        l_run = fmaf(l_run, alpha, sum);
+        m_run = m_new;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          o[j][0] *= alpha;
+          o[j][1] *= alpha;
+        }
+        uint32_t pa_[4] = {0u, 0u, 0u, 0u}, pl_[4] = {0u, 0u, 0u, 0u};
+        pack_split<T>(p0, p1, pa_[0], pl_[0]);
+        pack_split<T>(p2, p3, pa_[2], pl_[2]);
+        {
+          const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
+          const int col = (lane >> 4) * 8;
+#pragma unroll
+          for (int j = 0; j < NT; j += 2) {
+            uint32_t b[4];
+            ldmatrix_x4_trans(b, smem_addr(vtile + row * Cfg::PITCH + (j * 8 + col) * 2));
+            float d0[4] = {o[j][0], o[j][1], 0.f, 0.f};
+            float d1[4] = {o[j + 1][0], o[j + 1][1], 0.f, 0.f};
+            mma16816<T>(d0, pa_, b[0], b[1]);
+            mma16816<T>(d0, pl_, b[0], b[1]);
+            mma16816<T>(d1, pa_, b[2], b[3]);
+            mma16816<T>(d1, pl_, b[2], b[3]);
+            o[j][0] = d0[0];
+            o[j][1] = d0[1];
+            o[j + 1][0] = d1[0];
+            o[j + 1][1] = d1[1];
+          }
+        }
+        __syncwarp();
+        if (i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
+      }
+      if (!ok) {
+        if (lane == 0) {
+          atomicOr(a.err, PA_DEVERR_TIMEOUT);
+          s_abort = 1;
+        }
+        const int issued = min(nblk, i + NSTAGE);
+        for (int j = i; j < issued; ++j) {
+          const uint32_t k = k0 + j;
+          mbar_wait_bounded(smem_addr(&my_bars[k % NSTAGE]), (k / NSTAGE) & 1u);
+        }
+      } else {
+        fills = k0 + nblk;
+        if (row_ok) {
+          const int64_t sh = (int64_t)s * HQ + kvh * G + qrow;
+          const int d0 = (lane & 3) * 2;
+          if (!split) {
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            T* dst = static_cast<T*>(a.out) + sh * D + d0;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+              const uint32_t v = MmaType<T>::pack(o[j][0] * inv, o[j][1] * inv);
+              *reinterpret_cast<uint32_t*>(dst + j * 8) = v;
+            }
+          } else {
+            float* dst = a.part_acc + (sh * a.max_parts + p) * D + d0;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
+            if ((lane & 3) == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
+          }
+        }
+      }
+    }
+    if (split) {
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
+        __threadfence();
+        const int arrived = atomicAdd(cnt, 1) + 1;
+        s_merge = arrived == ni && !s_abort;
+        if (arrived == ni) *cnt = 0;
+      }
+      __syncthreads();
+      if (s_merge && kvh < HK) {
+        __threadfence();
+        for (int j = 0; j < G; ++j) merge_partitions<T, D>(a, (int64_t)s * HQ + kvh * G + j, np, lane);
+      }
+    }
+    __syncthreads();
+  }
+
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int done = atomicAdd(&a.plan->done_counter, 1);
+    if (done == (int)gridDim.x - 1) {
+      a.plan->work_counter = 0;
+      a.plan->done_counter = 0;
+      __threadfence();
+    }
+  }
+}
+
+}  // namespace pa

@@ -11,6 +11,7 @@
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "shared_prefix.cuh"
+#include "decode_gqa.cuh"
 #include "pagedattn.h"
 #include "status.h"
 
@@ -94,6 +95,38 @@ cudaError_t set_decode_attrs_all_groups() {
 // KV heads one work item covers, for G query heads per KV head.
 int rings_for(int G) { return warps_for(G) / G; }
 
+// Groups of 4 or 8 query heads on fp16/bf16 pools take the tensor-core
+// kernel (one warp per KV head); MHA, pairs (measured faster on CUDA cores)
+// and fp32 pools take the CUDA-core kernel.
+bool use_gqa_mma(const pa_pool* pool) { return pool->q_per_kv >= 4 && pool->dtype != PA_F32; }
+constexpr int kGqaStages = 2;
+
+int kv_heads_per_item(const pa_pool* pool) {
+  return use_gqa_mma(pool) ? GqaConfig<__half, 128, kGqaStages>::WARPS : rings_for(pool->q_per_kv);
+}
+
+template <typename T, int D>
+cudaError_t set_gqa_attrs() {
+  return cudaFuncSetAttribute(paged_decode_gqa_kernel<T, D, kGqaStages>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)GqaConfig<T, D, kGqaStages>::smem_bytes(kMaxPartition));
+}
+
+template <typename T, int D>
+cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
+  using Cfg = GqaConfig<T, D, kGqaStages>;
+  auto kernel = paged_decode_gqa_kernel<T, D, kGqaStages>;
+  const size_t smem = Cfg::smem_bytes(a.partition_size);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Cfg::THREADS, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = std::max(per_sm, 1);
+  const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
+  kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 // Once per device, with that device current: resolve the error word's device
 // address and raise the shared-memory limit of the decode kernels.
 pa_status device_state(DeviceState** out) {
@@ -115,7 +148,11 @@ pa_status device_state(DeviceState** out) {
                            set_decode_attrs_all_groups<__half, 64>(),
                            set_decode_attrs_all_groups<__half, 128>(),
                            set_decode_attrs_all_groups<__nv_bfloat16, 64>(),
-                           set_decode_attrs_all_groups<__nv_bfloat16, 128>()};
+                           set_decode_attrs_all_groups<__nv_bfloat16, 128>(),
+                           set_gqa_attrs<__half, 64>(),
+                           set_gqa_attrs<__half, 128>(),
+                           set_gqa_attrs<__nv_bfloat16, 64>(),
+                           set_gqa_attrs<__nv_bfloat16, 128>()};
     for (cudaError_t a : attrs)
       if (a != cudaSuccess) return cuda_fail(a, "cudaFuncSetAttribute");
     using Cfg = DecodeKernelCfg<__half, 128, 1>;
@@ -161,7 +198,8 @@ int total_parts(int maxL, int ps, int max_shared_blocks) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // H = query heads (partials are per query head); G = query heads per KV head.
-WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D, int G) {
+WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D, int G,
+                           int kv_per_item) {
   WorkspaceLayout w;
   size_t off = 0;
   w.header = off;
@@ -177,7 +215,7 @@ WorkspaceLayout layout_for(int64_t S, int64_t H, int64_t max_parts, int64_t D, i
   w.shared_of = off;
   off = align256(off + S * 4);
   w.merge_cnt = off;
-  off = align256(off + S * ((H / G + rings_for(G) - 1) / rings_for(G)) * 4);
+  off = align256(off + S * ((H / G + kv_per_item - 1) / kv_per_item) * 4);
   w.pairs = off;
   off = align256(off + S * max_parts * 8);
   w.part_ml = off;
@@ -333,7 +371,8 @@ pa_status pa_decode_shared_prefix_workspace_bytes(const pa_pool* pool, int32_t n
     return fail(PA_ERR_INVALID_ARG, "partition_size must be a multiple of 16 in [16, 4096]");
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
   *bytes = layout_for(num_seqs, (int64_t)pool->heads * pool->q_per_kv,
-                      total_parts(maxL, ps, max_shared_blocks), pool->head_dim, pool->q_per_kv)
+                      total_parts(maxL, ps, max_shared_blocks), pool->head_dim, pool->q_per_kv,
+                      kv_heads_per_item(pool))
                .total;
   return PA_OK;
 }
@@ -365,14 +404,14 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   if ((st = device_state(dev)) != PA_OK) return st;
   const int maxL = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
   const int G = pool->q_per_kv;
-  const int head_groups = (pool->heads + rings_for(G) - 1) / rings_for(G);
+  const int head_groups = (pool->heads + kv_heads_per_item(pool) - 1) / kv_heads_per_item(pool);
   const int ps = partition_size != 0
                      ? partition_size
                      : auto_partition(num_seqs, head_groups, maxL,
                                       (*dev)->num_sms * (*dev)->decode_ctas_per_sm);
   const int max_parts = total_parts(maxL, ps, max_shared_blocks);
-  const WorkspaceLayout w =
-      layout_for(num_seqs, (int64_t)pool->heads * G, max_parts, pool->head_dim, G);
+  const WorkspaceLayout w = layout_for(num_seqs, (int64_t)pool->heads * G, max_parts,
+                                       pool->head_dim, G, kv_heads_per_item(pool));
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(PA_ERR_WORKSPACE, "decode: workspace missing, not 256-byte aligned or too small");
   char* ws = static_cast<char*>(workspace);
@@ -411,6 +450,16 @@ pa_status launch_plan(const DecodeArgs& a, cudaStream_t s) {
 pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState& dev,
                      cudaStream_t s) {
   cudaError_t e;
+  if (use_gqa_mma(pool)) {
+    switch (pool->dtype * 1000 + pool->head_dim) {
+      case PA_F16 * 1000 + 64: e = launch_gqa<__half, 64>(a, dev, s); break;
+      case PA_F16 * 1000 + 128: e = launch_gqa<__half, 128>(a, dev, s); break;
+      case PA_BF16 * 1000 + 64: e = launch_gqa<__nv_bfloat16, 64>(a, dev, s); break;
+      case PA_BF16 * 1000 + 128: e = launch_gqa<__nv_bfloat16, 128>(a, dev, s); break;
+      default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
+    }
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode launch");
+  }
   switch (pool->dtype * 1000 + pool->head_dim) {
     case PA_F32 * 1000 + 64: e = launch_grouped<float, 64>(pool->q_per_kv, a, dev, s); break;
     case PA_F32 * 1000 + 128: e = launch_grouped<float, 128>(pool->q_per_kv, a, dev, s); break;

@@ -25,6 +25,7 @@
 
 #include "decode.cuh"
 #include "device_utils.cuh"
+#include "mma_utils.cuh"
 
 namespace pa {
 
@@ -36,70 +37,6 @@ struct SharedPrefixArgs {
   int32_t row_tiles;   // 64-row tiles per group (from the largest group)
   int32_t chunk_blocks;
 };
-
-template <typename T>
-struct MmaType;
-template <>
-struct MmaType<__half> {
-  __device__ __forceinline__ static uint32_t pack(float a, float b) {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-};
-template <>
-struct MmaType<__nv_bfloat16> {
-  __device__ __forceinline__ static uint32_t pack(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-};
-
-// d += a * b for one m16n8k16 tile (row-major A, column-major B, fp32 C/D).
-template <typename T>
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1);
-
-template <>
-__device__ __forceinline__ void mma16816<__half>(float* d, const uint32_t* a, uint32_t b0,
-                                                 uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-template <>
-__device__ __forceinline__ void mma16816<__nv_bfloat16>(float* d, const uint32_t* a, uint32_t b0,
-                                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t* r, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 template <int D>
 struct SharedPrefixConfig {
@@ -230,7 +167,7 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
       }
     }
     // online softmax on the fragments: c0,c1 -> row lane/4, c2,c3 -> row lane/4 + 8
-    uint32_t pa_[4];
+    uint32_t pa_[4], pl_[4];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       float x0 = s[0][2 * h2] * a.scale_log2, x1 = s[0][2 * h2 + 1] * a.scale_log2;
@@ -252,9 +189,10 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
         o[j][2 * h2] *= alpha;
         o[j][2 * h2 + 1] *= alpha;
       }
-      // P as the A fragment of the P.V product (k = tokens)
-      pa_[h2] = MmaType<T>::pack(p0, p1);      // row, tokens (lane%4)*2..+1
-      pa_[2 + h2] = MmaType<T>::pack(p2, p3);  // row, tokens 8 + (lane%4)*2..+1
+      // P as the A fragment of the P.V product (k = tokens), as a high part
+      // plus its rounding residual so bf16 operands keep the weights accurate
+      pack_split<T>(p0, p1, pa_[h2], pl_[h2]);          // row, tokens (lane%4)*2..+1
+      pack_split<T>(p2, p3, pa_[2 + h2], pl_[2 + h2]);  // row, tokens 8 + (lane%4)*2..+1
     }
     // O += P V: B fragments from V rows (tokens) by transposed ldmatrix
     {
@@ -265,7 +203,9 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
         uint32_t b[4];
         ldmatrix_x4_trans(b, smem_addr(vtile + row * Cfg::PITCH + (j * 8 + col) * 2));
         mma16816<T>(o[j], pa_, b[0], b[1]);
+        mma16816<T>(o[j], pl_, b[0], b[1]);
         mma16816<T>(o[j + 1], pa_, b[2], b[3]);
+        mma16816<T>(o[j + 1], pl_, b[2], b[3]);
       }
     }
   }

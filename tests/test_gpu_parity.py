@@ -397,7 +397,11 @@ def test_gqa_matches_oracle_and_replicated_mha(group, dtype, head_dim):
     ws_r = workspace_for(pool_r, len(lens), bt.shape[1])
     pa.pa_decode_attention(pool_r, q, dev(kr), dev(vr), bt, cl, case["scale"], out_r, ws_r)
     assert pa.pa_device_errors() == 0
-    assert torch.equal(out, out_r)
+    if dtype == np.float32:
+        assert torch.equal(out, out_r)  # same CUDA-core arithmetic per query head
+    else:
+        # fp16 groups run on tensor cores (P rounded to fp16 before P.V): same gate
+        assert_parity(out, out_r.double().cpu().numpy(), f"gqa x{group} vs repeated-KV MHA")
 
 
 @pytest.mark.parametrize("group", [4, 8])
@@ -429,3 +433,40 @@ def test_gqa_fused_append(group):
 
 
 TORCH = {np.float16: torch.float16, np.float32: torch.float32}
+
+
+@pytest.mark.parametrize("group", [2, 4, 8])
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_gqa_tensor_core_path_ragged_and_poisoned(group, head_dim):
+    """bf16 groups on the tensor-core path: lengths 0, 1 and ragged blocks,
+    NaN in every pool slot outside the cached tokens, several partition sizes."""
+    kv_heads = 3
+    lens = [0, 1, 2, 15, 16, 17, 100, 257, 1000]
+    case = syn.decode_case(51, lens, kv_heads, head_dim, np.float32, pool_fill="nan",
+                           num_pool_blocks=128, max_blocks=64)
+    rng = np.random.default_rng(52)
+    for s_, L in enumerate(lens):
+        slots = np.array([oracle.slot_of_c(case["block_tables"][s_], t) for t in range(L)],
+                         dtype=np.int32)
+        kn = rng.standard_normal((L, kv_heads, head_dim)).astype(np.float32)
+        vn = rng.standard_normal((L, kv_heads, head_dim)).astype(np.float32)
+        oracle.reshape_and_cache(kn, vn, slots, case["k_pool"], case["v_pool"])
+    qf = rng.standard_normal((len(lens), kv_heads * group, head_dim)).astype(np.float32)
+    kt = torch.from_numpy(case["k_pool"]).to(torch.bfloat16)
+    vt = torch.from_numpy(case["v_pool"]).to(torch.bfloat16)
+    qt = torch.from_numpy(qf).to(torch.bfloat16)
+    kb, vb, qb = (x.view(torch.int16).numpy().view(np.uint16) for x in (kt, vt, qt))
+    ref = oracle.decode_attention(qb, kb, vb, case["block_tables"], case["context_lens"],
+                                  case["scale"], dtype=oracle.BF16)
+    pool = pa.pa_pool_create(128, 16, kv_heads, head_dim, torch.bfloat16)
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    for ps in (0, 16, 96):
+        out = torch.empty((len(lens), kv_heads * group, head_dim), dtype=torch.bfloat16,
+                          device="cuda")
+        ws = workspace_for(pool, len(lens), bt.shape[1], 0, ps)
+        pa.pa_decode_attention(pool, qt.cuda(), kt.cuda(), vt.cuda(), bt, cl, case["scale"], out,
+                               ws, partition_size=ps)
+        assert pa.pa_device_errors() == 0
+        assert torch.isfinite(out.float()).all()
+        assert_parity(out, ref, f"gqa bf16 x{group} D={head_dim} ps={ps}")
