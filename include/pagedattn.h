@@ -245,6 +245,26 @@ pa_status pa_decode_attention_shared_prefix(
     size_t workspace_bytes, int32_t partition_size, void* stream);
 
 /*
+ * Paged prefill: many new query tokens per sequence attend causally to the
+ * sequence's paged cache ("PagedAttention" wiki mirror, "Formulació
+ * matemàtica": the block-wise form holds for every query token).  Sequence s
+ * has n_s = query_start[s+1] - query_start[s] new tokens, rows
+ * query_start[s].. of q and out ([T][heads * q_per_kv][head_dim]); they sit
+ * at positions context_lens[s] - n_s .. context_lens[s] - 1 and their K/V
+ * must already be in the pool (pa_reshape_and_cache).  Query i sees tokens
+ * 0..its position.  max_new_tokens bounds every n_s (launch sizing).
+ * Runs on tcgen05 tensor cores with TMEM accumulators; fp16/bf16 pools,
+ * head_dim 64 or 128.  A context length below n_s or above the table raises
+ * PA_DEVERR_CONTEXT_LEN and that sequence is skipped.
+ */
+pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* context_lens,
+                               const int32_t* query_start, int32_t num_seqs,
+                               int32_t max_new_tokens, int32_t max_context_len, float scale,
+                               void* out, void* stream);
+
+/*
  * Decode attention that allocates nothing.  Same computation, arguments and
  * errors as pa_decode_attention, minus the workspace: the plan and split-K
  * partials live in a static device buffer inside the library of

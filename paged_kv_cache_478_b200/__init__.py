@@ -88,6 +88,8 @@ def lib():
                                                   sz, i32, vp],
             "pa_find_shared_prefixes": [vp, i32, vp, i32, i32, i32, vp, vp, vp, P(i32), P(i32),
                                         P(i32)],
+            "pa_prefill_attention": [P(pa_pool), vp, vp, vp, vp, i32, vp, vp, i32, i32, i32,
+                                     ctypes.c_float, vp, vp],
             "pa_copy_blocks": [P(pa_pool), vp, vp, vp, i32, vp],
             "pa_device_errors": [vp, P(ctypes.c_uint32)],
             "pa_selftest_wait_timeout": [vp],
@@ -359,6 +361,27 @@ def pa_decode_attention_shared_prefix(pool, q, k_pool, v_pool, block_tables, con
         groups["max_group_size"], groups["max_shared_blocks"], max_context_len, float(scale),
         _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))
+
+
+def pa_prefill_attention(pool, q, k_pool, v_pool, block_tables, context_lens, query_start, scale,
+                         out, max_new_tokens, max_context_len=0, stream=None):
+    """Causal attention of many new tokens per sequence over the paged cache
+    (tcgen05).  q, out: [T, query heads, head_dim]; query_start: int32 [S+1]."""
+    torch = _torch()
+    S = context_lens.shape[0]
+    T = q.shape[0]
+    if tuple(q.shape) != (T, _q_heads(pool), pool.head_dim) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [tokens, query heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(query_start.shape) != (S + 1,):
+        raise ValueError("block_tables [S, max_blocks], context_lens [S], query_start [S+1]")
+    dt = _pool_torch_dtype(pool)
+    _check(lib().pa_prefill_attention(
+        ctypes.byref(pool), _dev_ptr(q, "q", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
+        _check_pool_tensor(pool, v_pool, "v_pool"),
+        _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev_ptr(context_lens, "context_lens", torch.int32),
+        _dev_ptr(query_start, "query_start", torch.int32), S, max_new_tokens, max_context_len,
+        float(scale), _dev_ptr(out, "out", dt), _stream(stream)))
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

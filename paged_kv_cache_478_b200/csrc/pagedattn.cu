@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "shared_prefix.cuh"
 #include "decode_gqa.cuh"
+#include "prefill.cuh"
 #include "pagedattn.h"
 #include "status.h"
 
@@ -106,6 +107,17 @@ int kv_heads_per_item(const pa_pool* pool) {
 }
 
 template <typename T, int D>
+size_t prefill_smem() {
+  return PrefillConfig<D, kSplitP<T>>::SMEM;
+}
+
+template <typename T, int D>
+cudaError_t set_prefill_attrs() {
+  return cudaFuncSetAttribute(paged_prefill_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)prefill_smem<T, D>());
+}
+
+template <typename T, int D>
 cudaError_t set_gqa_attrs() {
   return cudaFuncSetAttribute(paged_decode_gqa_kernel<T, D, kGqaStages>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -152,7 +164,11 @@ pa_status device_state(DeviceState** out) {
                            set_gqa_attrs<__half, 64>(),
                            set_gqa_attrs<__half, 128>(),
                            set_gqa_attrs<__nv_bfloat16, 64>(),
-                           set_gqa_attrs<__nv_bfloat16, 128>()};
+                           set_gqa_attrs<__nv_bfloat16, 128>(),
+                           set_prefill_attrs<__half, 64>(),
+                           set_prefill_attrs<__half, 128>(),
+                           set_prefill_attrs<__nv_bfloat16, 64>(),
+                           set_prefill_attrs<__nv_bfloat16, 128>()};
     for (cudaError_t a : attrs)
       if (a != cudaSuccess) return cuda_fail(a, "cudaFuncSetAttribute");
     using Cfg = DecodeKernelCfg<__half, 128, 1>;
@@ -663,6 +679,63 @@ pa_status pa_decode_attention_shared_prefix(
     if (e != cudaSuccess) return cuda_fail(e, "shared prefix launch");
   }
   return launch_run(pool, a, *dev, s);
+}
+
+pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* context_lens,
+                               const int32_t* query_start, int32_t num_seqs,
+                               int32_t max_new_tokens, int32_t max_context_len, float scale,
+                               void* out, void* stream) {
+  pa_status st = check_pool(pool);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || max_new_tokens < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "prefill: bad size");
+  if (num_seqs == 0 || max_new_tokens == 0) return PA_OK;
+  if (pool->dtype == PA_F32)
+    return fail(PA_ERR_UNSUPPORTED, "prefill: fp16 or bf16 pools only (tcgen05 kind::f16)");
+  st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
+  if (st != PA_OK) return st;
+  if (!context_lens || !query_start) return fail(PA_ERR_INVALID_ARG, "prefill: null pointer");
+  DeviceState* dev;
+  if ((st = device_state(&dev)) != PA_OK) return st;
+  PrefillArgs a{};
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start;
+  a.out = out;
+  a.err = dev->err;
+  a.num_blocks = pool->num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.heads = pool->heads;
+  a.q_per_kv = pool->q_per_kv;
+  a.max_context_len = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t qtiles = (max_new_tokens + 127) / 128;
+  const int64_t hq = (int64_t)pool->heads * pool->q_per_kv;
+  if (qtiles > INT32_MAX || hq > 65535 || num_seqs > 65535)
+    return fail(PA_ERR_INVALID_ARG, "prefill: grid too large");
+  const dim3 grid((unsigned)qtiles, (unsigned)hq, (unsigned)num_seqs);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = pool->dtype == PA_BF16;
+  if (pool->head_dim == 128) {
+    if (bf16)
+      paged_prefill_kernel<__nv_bfloat16, 128>
+          <<<grid, 128, prefill_smem<__nv_bfloat16, 128>(), s>>>(a);
+    else
+      paged_prefill_kernel<__half, 128><<<grid, 128, prefill_smem<__half, 128>(), s>>>(a);
+  } else {
+    if (bf16)
+      paged_prefill_kernel<__nv_bfloat16, 64><<<grid, 128, prefill_smem<__nv_bfloat16, 64>(), s>>>(a);
+    else
+      paged_prefill_kernel<__half, 64><<<grid, 128, prefill_smem<__half, 64>(), s>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "prefill launch");
 }
 
 pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,

@@ -1,0 +1,105 @@
+"""Paged prefill (tcgen05) against the oracle.
+
+Each new query token at position p must equal single-query attention over
+tokens 0..p of its sequence ("PagedAttention" wiki mirror, "Formulació
+matemàtica": the block-wise computation holds for every query), so the
+oracle is the pinned decode oracle run once per query token with
+context_len = p + 1 on the same block table."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_478_b200 as pa
+from tests.gpu_cases import assert_parity, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(seed, ctx_new, kv_heads, group, head_dim, dtype):
+    rng = np.random.default_rng(seed)
+    S = len(ctx_new)
+    lens = np.array([c for c, _ in ctx_new], dtype=np.int32)
+    news = np.array([n for _, n in ctx_new], dtype=np.int32)
+    need = [math.ceil(int(L) / 16) for L in lens]
+    nb = sum(need) + 5
+    maxb = max(need)
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((S, maxb), -1, dtype=np.int32)
+    pos = 0
+    for s, n in enumerate(need):
+        tables[s, :n] = perm[pos:pos + n]
+        pos += n
+    shape = (nb, kv_heads, 16, head_dim)
+    kf = rng.standard_normal(shape).astype(np.float32)
+    vf = rng.standard_normal(shape).astype(np.float32)
+    T = int(news.sum())
+    qf = rng.standard_normal((T, kv_heads * group, head_dim)).astype(np.float32)
+    qs = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    kt, vt, qt = (torch.from_numpy(x).to(tdt) for x in (kf, vf, qf))
+    if dtype == "bf16":
+        kh, vh, qh = (x.view(torch.int16).numpy().view(np.uint16) for x in (kt, vt, qt))
+        odt = oracle.BF16
+    else:
+        kh, vh, qh = (x.numpy() for x in (kt, vt, qt))
+        odt = None
+    # oracle: one decode row per query token, context = its position + 1
+    rows_t, rows_l = [], []
+    for s in range(S):
+        for i in range(int(news[s])):
+            rows_t.append(tables[s])
+            rows_l.append(int(lens[s]) - int(news[s]) + i + 1)
+    scale = 1 / math.sqrt(head_dim)
+    ref = oracle.decode_attention(qh, kh, vh, np.stack(rows_t), np.array(rows_l, np.int32),
+                                  scale, dtype=odt)
+    pool = pa.pa_pool_create(nb, 16, kv_heads, head_dim, tdt)
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    return dict(pool=pool, q=qt.cuda(), k=kt.cuda(), v=vt.cuda(), tables=dev(tables),
+                lens=dev(lens), qs=dev(qs), max_new=int(news.max()), ref=ref, scale=scale)
+
+
+CASES = [(1, 1), (17, 17), (200, 64), (300, 300), (1000, 129), (128, 128), (2048, 256),
+         (700, 1), (45, 13)]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("head_dim", [128, 64])
+@pytest.mark.parametrize("group", [1, 4])
+def test_prefill_matches_the_oracle(dtype, head_dim, group):
+    c = _case(70 + group, CASES, 2, group, head_dim, dtype)
+    out = torch.empty_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], c["qs"],
+                            c["scale"], out, c["max_new"])
+    assert pa.pa_device_errors() == 0
+    assert torch.isfinite(out.float()).all()
+    assert_parity(out, c["ref"], f"prefill {dtype} D={head_dim} G={group}")
+
+
+def test_prefill_single_new_token_matches_decode():
+    """n = 1 is decode: the two paths agree within the gate."""
+    ctx = [(1, 1), (16, 1), (17, 1), (513, 1), (2000, 1)]
+    c = _case(80, ctx, 4, 1, 128, "f16")
+    out = torch.empty_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], c["qs"],
+                            c["scale"], out, 1)
+    d_out = torch.empty_like(c["q"])
+    ws = torch.empty(pa.pa_decode_workspace_bytes(c["pool"], len(ctx), c["tables"].shape[1]),
+                     dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], c["scale"],
+                           d_out, ws)
+    assert pa.pa_device_errors() == 0
+    assert_parity(out, c["ref"], "prefill n=1")
+    assert_parity(d_out, c["ref"], "decode")
+
+
+def test_prefill_rejects_a_context_shorter_than_its_new_tokens():
+    c = _case(81, [(40, 20), (30, 10)], 2, 1, 64, "f16")
+    bad = torch.tensor([40, 5], dtype=torch.int32, device="cuda")  # 5 < 10 new tokens
+    out = torch.zeros_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], bad, c["qs"],
+                            c["scale"], out, 20)
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
+    assert_parity(out[:20], c["ref"][:20], "the valid sequence still runs")
