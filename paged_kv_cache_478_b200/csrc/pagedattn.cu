@@ -1,6 +1,8 @@
 // C ABI of libpagedattn.so: host-side validation, per-device set-up and
 // kernel launches.  Declarations and argument contracts: include/pagedattn.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cmath>
@@ -41,6 +43,8 @@ struct DeviceState {
   uint32_t* err = nullptr;  // device address of g_device_errors
   int num_sms = 0;
   int decode_ctas_per_sm = 1;  // resident decode CTAs per SM (fp16, head_dim 128 kernel)
+  // driver's tensor-map encoder, resolved through the runtime (no libcuda link)
+  PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
 };
 
 std::mutex g_mutex;
@@ -111,6 +115,37 @@ size_t prefill_smem() {
   return PrefillConfig<D, kSplitP<T>>::SMEM;
 }
 
+// K or V pool as a 2-D tensor [num_blocks * heads * 16 rows][head_dim] with a
+// {64, 16} box (one physical block, one 64-wide slice of head_dim) and
+// 128-byte swizzle: the prefill kernel's tile layout.
+pa_status encode_pool_map(const DeviceState& dev, CUtensorMap* map, const void* base,
+                          const pa_pool* pool) {
+  const cuuint64_t dims[2] = {(cuuint64_t)pool->head_dim,
+                              (cuuint64_t)pool->num_blocks * pool->heads * kBlock};
+  const cuuint64_t strides[1] = {(cuuint64_t)pool->head_dim * pool->elem_bytes};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)kBlock};
+  const cuuint32_t elem_strides[2] = {1u, 1u};
+  const CUresult r = dev.encode_tiled(
+      map, pool->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+      2, const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    std::snprintf(buf, sizeof buf, "prefill: cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return fail(PA_ERR_CUDA, buf);
+  }
+  return PA_OK;
+}
+
+template <typename T, int D>
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& k, const CUtensorMap& v,
+                           dim3 grid, cudaStream_t s) {
+  paged_prefill_kernel<T, D><<<grid, PrefillConfig<D, kSplitP<T>>::THREADS, prefill_smem<T, D>(),
+                               s>>>(a, k, v);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t set_prefill_attrs() {
   return cudaFuncSetAttribute(paged_prefill_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -155,6 +190,13 @@ pa_status device_state(DeviceState** out) {
     st.err = static_cast<uint32_t*>(p);
     e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPointByVersion");
+    if (q != cudaDriverEntryPointSuccess || !fn)
+      return fail(PA_ERR_CUDA, "driver has no cuTensorMapEncodeTiled");
+    st.encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     cudaError_t attrs[] = {set_decode_attrs_all_groups<float, 64>(),
                            set_decode_attrs_all_groups<float, 128>(),
                            set_decode_attrs_all_groups<__half, 64>(),
@@ -701,7 +743,6 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
   if ((st = device_state(&dev)) != PA_OK) return st;
   PrefillArgs a{};
   a.q = q;
-  a.k_pool = k_pool;
   a.v_pool = v_pool;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
@@ -715,26 +756,27 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
   a.q_per_kv = pool->q_per_kv;
   a.max_context_len = resolve_max_context(pool, max_blocks_per_seq, max_context_len);
   a.scale_log2 = scale * 1.4426950408889634f;
-  const int64_t qtiles = (max_new_tokens + 127) / 128;
+  const int64_t pairs = (max_new_tokens + 255) / 256;  // two 128-query tiles per CTA
   const int64_t hq = (int64_t)pool->heads * pool->q_per_kv;
-  if (qtiles > INT32_MAX || hq > 65535 || num_seqs > 65535)
+  if (pairs > INT32_MAX || hq > 65535 || num_seqs > 65535)
     return fail(PA_ERR_INVALID_ARG, "prefill: grid too large");
-  const dim3 grid((unsigned)qtiles, (unsigned)hq, (unsigned)num_seqs);
+  if ((int64_t)pool->num_blocks * pool->heads * kBlock > INT32_MAX)
+    return fail(PA_ERR_INVALID_ARG, "prefill: pool rows exceed the tensor-copy coordinate range");
+  a.q_pairs = (int32_t)pairs;
+  CUtensorMap tk, tv;
+  if ((st = encode_pool_map(*dev, &tk, k_pool, pool)) != PA_OK ||
+      (st = encode_pool_map(*dev, &tv, v_pool, pool)) != PA_OK)
+    return st;
+  const dim3 grid((unsigned)pairs, (unsigned)hq, (unsigned)num_seqs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = pool->dtype == PA_BF16;
-  if (pool->head_dim == 128) {
-    if (bf16)
-      paged_prefill_kernel<__nv_bfloat16, 128>
-          <<<grid, 128, prefill_smem<__nv_bfloat16, 128>(), s>>>(a);
-    else
-      paged_prefill_kernel<__half, 128><<<grid, 128, prefill_smem<__half, 128>(), s>>>(a);
-  } else {
-    if (bf16)
-      paged_prefill_kernel<__nv_bfloat16, 64><<<grid, 128, prefill_smem<__nv_bfloat16, 64>(), s>>>(a);
-    else
-      paged_prefill_kernel<__half, 64><<<grid, 128, prefill_smem<__half, 64>(), s>>>(a);
-  }
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (pool->head_dim == 128)
+    e = bf16 ? launch_prefill<__nv_bfloat16, 128>(a, tk, tv, grid, s)
+             : launch_prefill<__half, 128>(a, tk, tv, grid, s);
+  else
+    e = bf16 ? launch_prefill<__nv_bfloat16, 64>(a, tk, tv, grid, s)
+             : launch_prefill<__half, 64>(a, tk, tv, grid, s);
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "prefill launch");
 }
 

@@ -6,24 +6,31 @@
 // applies to every query; with 128 queries a tile the two products are dense
 // contractions, S = Q.K^T and O = P.V.
 //
-// One CTA = (sequence, query head, tile of 128 new queries); 4 warps, thread
-// r owns query row r.  Per 64-key tile:
-//   * all threads stage K and V rows from their physical blocks with cp.async
-//     into 128-byte-swizzled tiles (two stages), rows past the context are
-//     zeroed;
-//   * thread 0 issues S = Q.K^T (M=128, N=64, K=head_dim in steps of 16) into
-//     TMEM and commits to an mbarrier;
-//   * each thread reads its row of S from TMEM, applies the causal mask and
-//     the online softmax in fp32 (log2 domain), rescales its row of O in TMEM
-//     when the running max moved, and writes its row of P (fp16/bf16) into a
-//     swizzled shared tile;
-//   * thread 0 issues O += P.V (M=128, N=head_dim, K=64) into TMEM.
+// One CTA = (sequence, query head, 256 new queries as two 128-row tiles) with
+// specialised warps:
+//   * warps 0-3 and 4-7: two softmax warpgroups, one per query tile; thread r
+//     of a group owns query row r (TMEM lane r).  Each reads its row of S from
+//     TMEM, applies the causal mask and the online softmax in fp32 (log2
+//     domain) and writes its row of P (fp16/bf16) into a swizzled shared tile;
+//   * warp 8: the loader.  It streams the paged K and V rows of each 64-key
+//     tile with TMA tensor copies (one 16-row box per physical block and
+//     64-wide slice of head_dim, hardware 128-byte swizzle) into a ring of
+//     K/V stages; the valid V rows of a partly filled last block are copied
+//     by its lanes and the V rows past the context are zeroed;
+//   * warp 9: one thread issues the tensor-core products into TMEM and commits
+//     them to mbarriers.
+// The two query tiles share every K/V stage and take turns on the tensor core:
+// while one group runs its softmax, the MMA unit computes the other group's
+// P.V and next S.  The running max is only moved (and the row of O in TMEM
+// rescaled) when a score exceeds it by more than 2^8, which keeps every
+// weight at most 256 and makes the rescale rare.
 // Shared-memory operands are described by SW128 matrix descriptors (K-major
-// for Q, K and P; MN-major for V).  TMEM holds S (64 columns) and O
-// (head_dim columns); the CTA allocates 256 columns and frees them on every
-// exit path.  Every wait is bounded.
+// for Q, K and P; MN-major for V).  Every wait is bounded; a wait that gives
+// up stops the CTA's other roles, lets every copy and product already issued
+// land, frees TMEM and reports PA_DEVERR_TIMEOUT.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -38,9 +45,8 @@
 namespace pa {
 
 struct PrefillArgs {
-  const void* q;            // [T][HQ][D]
-  const void* k_pool;
-  const void* v_pool;
+  const void* q;                // [T][HQ][D]
+  const void* v_pool;           // rows of a partly filled last block are copied directly
   const int32_t* block_tables;
   const int32_t* context_lens;  // [S] tokens cached, new ones included
   const int32_t* query_start;   // [S+1] CSR: new tokens of s are rows query_start[s].. of q/out
@@ -52,6 +58,7 @@ struct PrefillArgs {
   int32_t heads;     // KV heads
   int32_t q_per_kv;  // query heads per KV head
   int32_t max_context_len;
+  int32_t q_pairs;   // 256-query units per sequence in the grid (blockIdx.x range)
   float scale_log2;
 };
 
@@ -60,27 +67,36 @@ struct PrefillArgs {
 // significand); fp16's 11 bits keep the result inside the parity gate alone.
 template <int D, bool SPLIT_P>
 struct PrefillConfig {
-  static constexpr int BM = 128;  // queries per CTA (TMEM lanes)
-  static constexpr int BN = 64;   // keys per tile
-  static constexpr int KB = D / 64;                 // 128-byte K-blocks across head_dim
+  static constexpr int BM = 128;        // query rows per tile (TMEM lanes)
+  static constexpr int QT = 2;          // query tiles per CTA (softmax warpgroups)
+  static constexpr int BN = 64;         // keys per tile
+  static constexpr int KB = D / 64;     // 128-byte K-blocks across head_dim
+  static constexpr int NS = 3;          // K/V ring stages
+  static constexpr int NP = SPLIT_P ? 2 : 1;
+  static constexpr int LOAD_WARP = 8, MMA_WARP = 9;
+  static constexpr int THREADS = 320;
   static constexpr int Q_BYTES = KB * BM * 128;
-  static constexpr int KV_BYTES = KB * BN * 128;    // one of K or V
-  static constexpr int P_BYTES = BM * 128;          // BM rows x 64 keys
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + Q_BYTES;    // [stage][K|V]
-  static constexpr int OFF_P = OFF_KV + 2 * 2 * KV_BYTES;      // P (high part)
-  static constexpr int OFF_PL = OFF_P + P_BYTES;               // P residual (SPLIT_P)
-  static constexpr int OFF_BAR = OFF_PL + (SPLIT_P ? P_BYTES : 0);  // 2 mbarriers + TMEM address
-  // The dynamic window starts 1024-byte aligned when the kernel has no static
-  // shared variables (checked at run time), so two CTAs fit per SM.
-  static constexpr size_t SMEM = OFF_BAR + 64;
-  static constexpr int TMEM_COLS = 256;             // S: 64 columns, O: D columns
-  static constexpr int S_COL = 0;
-  static constexpr int O_COL = 64;
+  static constexpr int KV_BYTES = KB * BN * 128;   // one of K or V
+  static constexpr int P_BYTES = BM * 128;         // BM rows x 64 keys
+  static constexpr int OFF_Q = 0;                               // [tile]
+  static constexpr int OFF_KV = OFF_Q + QT * Q_BYTES;           // [stage][K|V]
+  static constexpr int OFF_P = OFF_KV + NS * 2 * KV_BYTES;      // [tile][high|residual]
+  static constexpr int OFF_BAR = OFF_P + QT * NP * P_BYTES;
+  // mbarriers: q_full[2], full[NS], empty[NS], s_full[2], p_full[2], o_done[2], fin
+  static constexpr int BAR_Q = 0, BAR_FULL = 2, BAR_EMPTY = 2 + NS, BAR_S = 2 + 2 * NS,
+                       BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_FIN = BAR_O + 2,
+                       NBARS = BAR_FIN + 1;
+  static constexpr int OFF_SLOT = OFF_BAR + NBARS * 8;  // TMEM address, abort flag
+  // + 1 KB so the swizzled tiles can start on a 1024-byte boundary
+  static constexpr size_t SMEM = OFF_SLOT + 16 + 1024;
+  static constexpr int S_COL0 = 0;                  // S of tile w at w * BN
+  static constexpr int O_COL0 = 2 * BN;             // O of tile w at O_COL0 + w * D
+  static constexpr int TMEM_COLS = (O_COL0 + 2 * D) <= 256 ? 256 : 512;
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
-// ---- tcgen05 / descriptor helpers ------------------------------------------------
+// ---- tcgen05 / TMA helpers -------------------------------------------------------
 
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading
 // and stride byte offsets (16-byte units), version 1, layout type 2.
@@ -122,7 +138,8 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+// 32 consecutive TMEM columns of this warp's 32 lanes into v (no wait).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float* v) {
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -133,9 +150,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  tmem_ld32_nowait(taddr, v);
+  tmem_wait_ld();
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
@@ -157,8 +181,48 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2-D tiled tensor copy global -> shared (no multicast), completing its bytes
+// on `bar`.  x is the innermost coordinate (elements), y the row.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait that also gives up once another role raised the abort flag.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                   const volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) return false;
+  }
+}
+
+// The same for every lane of a warp: the warp goes on only if all its lanes saw
+// the phase complete, so a give-up never splits a warp.
+__device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                   const volatile int* abort_flag) {
+  return __all_sync(kFullMask, mbar_wait_or_abort(bar, parity, abort_flag));
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile whose
-// rows are 128 bytes (one K-block).
+// rows are 128 bytes (one K-block).  The TMA copies with 128-byte swizzle
+// produce the same placement for boxes that start 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
@@ -166,25 +230,27 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 template <typename T>
 constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
 
+// tm_k, tm_v: K and V pools viewed as [num_blocks * heads * 16 rows][head_dim],
+// box {64, 16} (one physical block, one 64-wide slice), 128-byte swizzle.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) paged_prefill_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(320, 1)
+    paged_prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   using Cfg = PrefillConfig<D, kSplitP<T>>;
-  constexpr int BM = Cfg::BM, BN = Cfg::BN;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, KB = Cfg::KB, NS = Cfg::NS;
   constexpr uint32_t IDESC_S = f16_idesc(BM, BN, kBf16, false);
   constexpr uint32_t IDESC_PV = f16_idesc(BM, D, kBf16, true);
 
   extern __shared__ __align__(1024) uint8_t prefill_smem[];
-  uint8_t* smem = prefill_smem;
+  uint8_t* smem = prefill_smem + ((1024u - (smem_addr(prefill_smem) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
 
-  const int qt = blockIdx.x, hq = blockIdx.y, s = blockIdx.z;
-  if (smem_addr(smem) & 1023u) {  // the swizzled tiles need a 1024-byte aligned base
-    if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_TIMEOUT);
-    return;
-  }
+  // heaviest query pairs (latest positions, most keys) first
+  const int qt = a.q_pairs - 1 - (int)blockIdx.x, hq = blockIdx.y, s = blockIdx.z;
   const int q0 = a.query_start[s];
   const int n = a.query_start[s + 1] - q0;
-  if (n <= 0 || qt * BM >= n) return;
+  if (n <= 0 || qt * 2 * BM >= n) return;
   const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
   const int L = a.context_lens[s];
   if (L < n || L > cap) {  // the new tokens must be in the cache
@@ -192,19 +258,17 @@ __global__ void __launch_bounds__(128) paged_prefill_kernel(PrefillArgs a) {
     return;
   }
   const int G = a.q_per_kv, HQ = a.heads * G, kvh = hq / G;
-  const int row = threadIdx.x, warp = row >> 5;
-  const int qi = qt * BM + row;
-  const bool row_valid = qi < n;
-  const int pos = L - n + qi;                               // this query's position
-  const int last_pos = L - n + min(n, (qt + 1) * BM) - 1;  // last query of the tile
-  const int nkt = (last_pos + BN) / BN;                     // key tiles to visit
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has1 = qt * 2 * BM + BM < n;  // second query tile holds queries
+  // key tiles each query tile visits (up to its last query's position)
+  const int nkt0 = (L - n + min(n, qt * 2 * BM + BM) - 1 + BN) / BN;
+  const int nkt1 = has1 ? (L - n + min(n, qt * 2 * BM + 2 * BM) - 1 + BN) / BN : 0;
+  const int nkt = has1 ? nkt1 : nkt0;
 
-  uint8_t* sQ = smem + Cfg::OFF_Q;
-  uint8_t* sP = smem + Cfg::OFF_P;
-  uint8_t* sPL = smem + Cfg::OFF_PL;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_BAR + 16);
-  const uint32_t bar_s = smem_addr(&bars[0]), bar_pv = smem_addr(&bars[1]);
+  auto bar = [&](int i) { return smem_addr(&bars[i]); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_SLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_SLOT + 4);
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -213,202 +277,318 @@ __global__ void __launch_bounds__(128) paged_prefill_kernel(PrefillArgs a) {
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (threadIdx.x == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_pv, 1);
+  if (threadIdx.x == 32) {
+    mbar_init(bar(Cfg::BAR_Q + 0), BM);
+    mbar_init(bar(Cfg::BAR_Q + 1), BM);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar(Cfg::BAR_FULL + i), 1);
+      mbar_init(bar(Cfg::BAR_EMPTY + i), 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(Cfg::BAR_S + w), 1);
+      mbar_init(bar(Cfg::BAR_P + w), BM);
+      mbar_init(bar(Cfg::BAR_O + w), 1);
+    }
+    mbar_init(bar(Cfg::BAR_FIN), 1);
+    *abort_flag = 0;
     mbar_init_fence();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
 
-  // ---- Q tile: row r = query qt*BM + r, zero past the new tokens -------------
-  {
-    constexpr int CH = D / 8;  // 16-byte chunks per row
-    for (int idx = threadIdx.x; idx < BM * CH; idx += blockDim.x) {
-      const int r = idx / CH, c = idx % CH;
-      uint8_t* dst = sQ + (c >> 3) * (BM * 128) + sw128_off(r, c & 7);
-      if (qt * BM + r < n) {
-        const T* src = static_cast<const T*>(a.q) + ((int64_t)(q0 + qt * BM + r) * HQ + hq) * D + c * 8;
-        cp_async16(smem_addr(dst), src);
-      } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      }
+  auto give_up = [&]() {
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      atomicOr(a.err, PA_DEVERR_TIMEOUT);
     }
-  }
-  const int32_t* table = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-  const int64_t tile_elems = (int64_t)kBlock * D;
-  const int64_t block_elems = (int64_t)a.heads * tile_elems;
-  // stage K/V rows of key tile j (tokens j*BN ..): rows at or past L are zeroed
-  auto load_kv = [&](int j, int stage) {
-    uint8_t* sK = smem + Cfg::OFF_KV + stage * 2 * Cfg::KV_BYTES;
-    uint8_t* sV = sK + Cfg::KV_BYTES;
-    constexpr int CH = D / 8;
-    for (int idx = threadIdx.x; idx < BN * CH; idx += blockDim.x) {
-      const int r = idx / CH, c = idx % CH;
-      const int t = j * BN + r;
-      const uint32_t off = (c >> 3) * (BN * 128) + sw128_off(r, c & 7);
-      if (t < L) {
-        int32_t blk = table[t / kBlock];
+  };
+
+  if (warp == Cfg::LOAD_WARP) {
+    // ---- loader: K and V of key tile j into stage j % NS ------------------------
+    const int32_t* table = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+    int issued = 0;
+    for (int j = 0; j < nkt; ++j) {
+      const int st = j % NS;
+      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_EMPTY + st), ((j / NS) - 1) & 1, abort_flag)) {
+        give_up();
+        break;
+      }
+      const uint32_t sK = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES;
+      const uint32_t sV = sK + Cfg::KV_BYTES;
+      uint8_t* gV = smem + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES;
+      // V rows at or past the context are zeroed (their weights are zero, but
+      // stale bits may be NaN); K rows there are masked out of S by selection.
+      // A partly filled last block's valid V rows are copied by the lanes, so
+      // every tensor copy moves a whole block.
+      const int valid_in_tile = min(BN, L - j * BN);
+      const int nblk = (valid_in_tile + kBlock - 1) / kBlock;  // blocks holding tokens
+      const bool partial = valid_in_tile < nblk * kBlock;
+      auto block_of = [&](int i) {
+        int32_t blk = table[j * (BN / kBlock) + i];
         if (blk < 0 || blk >= a.num_blocks) {
           atomicOr(a.err, PA_DEVERR_BLOCK_ID);
           blk = 0;
         }
-        const int64_t e = blk * block_elems + kvh * tile_elems + (int64_t)(t % kBlock) * D + c * 8;
-        cp_async16(smem_addr(sK + off), static_cast<const T*>(a.k_pool) + e);
-        cp_async16(smem_addr(sV + off), static_cast<const T*>(a.v_pool) + e);
-      } else {
-        *reinterpret_cast<uint4*>(sK + off) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sV + off) = make_uint4(0, 0, 0, 0);
+        return blk;
+      };
+      if (valid_in_tile < BN) {
+        const int r_lo = partial ? (nblk - 1) * kBlock : valid_in_tile;
+        const T* src = nullptr;
+        if (partial)
+          src = static_cast<const T*>(a.v_pool) +
+                (((int64_t)block_of(nblk - 1) * a.heads + kvh) * kBlock) * D;
+        for (int idx = lane; idx < (BN - r_lo) * KB * 8; idx += 32) {
+          const int r = r_lo + idx / (KB * 8), c = idx % (KB * 8);
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (r < valid_in_tile)
+            v = *reinterpret_cast<const uint4*>(src + (int64_t)(r - r_lo) * D + c * 8);
+          *reinterpret_cast<uint4*>(gV + (c >> 3) * (BN * 128) + sw128_off(r, c & 7)) = v;
+        }
+        fence_proxy_async_shared();
       }
-    }
-  };
-  load_kv(0, 0);
-  cp_async_commit();  // group 0: Q + key tile 0
-
-  float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true;
-  int last_s = -1, last_pv = -1;  // last tiles whose products were issued (uniform)
-  for (int j = 0; j < nkt; ++j) {
-    const int stage = j & 1;
-    if (j >= 1) {
-      // O += P.V of tile j-1 done: O is stable, P and stage (j+1)&1 are free
-      ok = mbar_wait_bounded(bar_pv, (j - 1) & 1);
-      if (!__syncthreads_and(ok)) break;
-      tc_fence_after();
-    }
-    if (j + 1 < nkt) load_kv(j + 1, stage ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();          // this thread's copies of tile j have landed
-    fence_proxy_async_shared();  // ... and are visible to the tensor core
-    __syncthreads();
-
-    uint8_t* sK = smem + Cfg::OFF_KV + stage * 2 * Cfg::KV_BYTES;
-    uint8_t* sV = sK + Cfg::KV_BYTES;
-    if (threadIdx.x == 0) {
-      tc_fence_after();
+      __syncwarp();
+      if (lane == 0) {
+        const int nfull_v = partial ? nblk - 1 : nblk;
+        const uint32_t bytes = (uint32_t)(nblk + nfull_v) * KB * kBlock * 128;
+        mbar_arrive_expect_tx(bar(Cfg::BAR_FULL + st), bytes);
+        for (int i = 0; i < nblk; ++i) {
+          const int row0 = (int)(((int64_t)block_of(i) * a.heads + kvh) * kBlock);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t kofs = (kk & 3) * 32;  // 16 elements further along the 128-byte row
-        const uint64_t ad = sw128_desc(smem_addr(sQ + (kk >> 2) * (BM * 128)) + kofs, 16, 1024);
-        const uint64_t bd = sw128_desc(smem_addr(sK + (kk >> 2) * (BN * 128)) + kofs, 16, 1024);
-        umma_f16(tmem + Cfg::S_COL, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(bar_s);
-    }
-    last_s = j;
-    ok = mbar_wait_bounded(bar_s, j & 1);
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
-
-    // ---- this row's scores, causal mask, online softmax -----------------------
-    float sc[BN];
-    tmem_ld32(tmem + lane_base + Cfg::S_COL, sc);
-    tmem_ld32(tmem + lane_base + Cfg::S_COL + 32, sc + 32);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < BN; ++c) {
-      const int t = j * BN + c;
-      sc[c] = (row_valid && t <= pos) ? sc[c] * a.scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sc[c]);
-    }
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = m_new == -INFINITY ? 1.f : exp2f(m_run - m_new);
-    float sum = 0.f;
-#pragma unroll
-    for (int c = 0; c < BN; ++c) {
-      sc[c] = m_new == -INFINITY ? 0.f : exp2f(sc[c] - m_new);
-      sum += sc[c];
-    }
-    l_run = fmaf(l_run, alpha, sum);
-    m_run = m_new;
-    // rescale this row of O when the running max moved (the whole warp takes
-    // part in the TMEM access if any of its rows needs it)
-    if (j >= 1 && __any_sync(kFullMask, alpha != 1.f)) {
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + Cfg::O_COL + c0, o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-        tmem_st32(tmem + lane_base + Cfg::O_COL + c0, o);
-      }
-    }
-    // this row of P into the swizzled A tile (64 keys = 8 chunks of 16 bytes)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4 v, r;
-      if constexpr (Cfg::OFF_PL != Cfg::OFF_BAR) {  // SPLIT_P
-        pack_split<T>(sc[8 * c + 0], sc[8 * c + 1], v.x, r.x);
-        pack_split<T>(sc[8 * c + 2], sc[8 * c + 3], v.y, r.y);
-        pack_split<T>(sc[8 * c + 4], sc[8 * c + 5], v.z, r.z);
-        pack_split<T>(sc[8 * c + 6], sc[8 * c + 7], v.w, r.w);
-        *reinterpret_cast<uint4*>(sPL + sw128_off(row, c)) = r;
-      } else {
-        v.x = MmaType<T>::pack(sc[8 * c + 0], sc[8 * c + 1]);
-        v.y = MmaType<T>::pack(sc[8 * c + 2], sc[8 * c + 3]);
-        v.z = MmaType<T>::pack(sc[8 * c + 4], sc[8 * c + 5]);
-        v.w = MmaType<T>::pack(sc[8 * c + 6], sc[8 * c + 7]);
-      }
-      *reinterpret_cast<uint4*>(sP + sw128_off(row, c)) = v;
-    }
-    fence_proxy_async_shared();
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint64_t ad = sw128_desc(smem_addr(sP) + kk * 32, 16, 1024);
-        // V is MN-major: 64-dim blocks LBO apart, 8-key groups 1024 bytes apart
-        const uint64_t bd = sw128_desc(smem_addr(sV) + kk * 2048, BN * 128, 1024);
-        umma_f16(tmem + Cfg::O_COL, ad, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-        if constexpr (Cfg::OFF_PL != Cfg::OFF_BAR) {
-          const uint64_t adl = sw128_desc(smem_addr(sPL) + kk * 32, 16, 1024);
-          umma_f16(tmem + Cfg::O_COL, adl, bd, IDESC_PV, 1u);
+          for (int kb = 0; kb < KB; ++kb) {
+            const uint32_t o = kb * (BN * 128) + i * (kBlock * 128);
+            tma_load_2d(sK + o, &tm_k, kb * 64, row0, bar(Cfg::BAR_FULL + st));
+            if (i < nfull_v) tma_load_2d(sV + o, &tm_v, kb * 64, row0, bar(Cfg::BAR_FULL + st));
+          }
         }
       }
-      umma_commit(bar_pv);
+      issued = j + 1;
     }
-    last_pv = j;
-  }
-  if (ok) ok = mbar_wait_bounded(bar_pv, (nkt - 1) & 1);
-  ok = __syncthreads_and(ok);
-  if (!ok) {
-    // a wait gave up: let the products already issued land (bounded) before
-    // the shared memory and TMEM are released
-    if (last_s >= 0) mbar_wait_bounded(bar_s, last_s & 1);
-    if (last_pv >= 0) mbar_wait_bounded(bar_pv, last_pv & 1);
-  }
-  tc_fence_after();
+    // let the copies of the last stages land before the CTA releases its memory
+    if (lane == 0)
+      for (int j = max(0, issued - NS); j < issued; ++j)
+        mbar_wait_bounded(bar(Cfg::BAR_FULL + j % NS), (j / NS) & 1);
+  } else if (warp == Cfg::MMA_WARP) {
+    // ---- MMA issue ------------------------------------------------------------------
+    if (lane == 0) {
+      auto issue_s = [&](int w, int st) {
+        const uint32_t qa = sbase + Cfg::OFF_Q + w * Cfg::Q_BYTES;
+        const uint32_t ka = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kofs = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint32_t kofs_b = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          umma_f16(tmem + Cfg::S_COL0 + w * BN, sw128_desc(qa + kofs, 16, 1024),
+                   sw128_desc(ka + kofs_b, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int w, int st, bool first) {
+        const uint32_t pa = sbase + Cfg::OFF_P + w * Cfg::NP * Cfg::P_BYTES;
+        const uint32_t va = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // V is MN-major: 64-dim blocks LBO apart, 8-key groups 1024 bytes apart
+          const uint64_t bd = sw128_desc(va + kk * 2048, BN * 128, 1024);
+          umma_f16(tmem + Cfg::O_COL0 + w * D, sw128_desc(pa + kk * 32, 16, 1024), bd, IDESC_PV,
+                   (!first || kk > 0) ? 1u : 0u);
+          if constexpr (Cfg::NP == 2)
+            umma_f16(tmem + Cfg::O_COL0 + w * D,
+                     sw128_desc(pa + Cfg::P_BYTES + kk * 32, 16, 1024), bd, IDESC_PV, 1u);
+        }
+      };
+      int ready = -1;  // last key tile whose stage was seen full
+      auto wait_kv = [&](int j) {
+        if (j <= ready) return true;
+        if (!mbar_wait_or_abort(bar(Cfg::BAR_FULL + j % NS), (j / NS) & 1, abort_flag)) return false;
+        ready = j;
+        tc_fence_after();
+        return true;
+      };
+      bool ok = mbar_wait_or_abort(bar(Cfg::BAR_Q + 0), 0, abort_flag) && wait_kv(0) &&
+                (!has1 || mbar_wait_or_abort(bar(Cfg::BAR_Q + 1), 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(bar(Cfg::BAR_S + 0));
+        if (has1) {
+          issue_s(1, 0);
+          umma_commit(bar(Cfg::BAR_S + 1));
+        }
+      }
+      for (int j = 0; ok && j < nkt; ++j) {
+        const int st = j % NS;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int nk = w == 0 ? nkt0 : nkt1;
+          if (j >= nk) continue;
+          if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + w), j & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(w, st, j == 0);
+          if (j == nk - 1) {
+            umma_commit(bar(Cfg::BAR_O + w));
+          } else {
+            if (!(ok = wait_kv(j + 1))) break;
+            issue_s(w, (j + 1) % NS);
+            umma_commit(bar(Cfg::BAR_S + w));
+          }
+        }
+        if (ok) umma_commit(bar(Cfg::BAR_EMPTY + st));
+      }
+      if (!ok) give_up();
+      // every product issued has completed before TMEM and shared memory go
+      umma_commit(bar(Cfg::BAR_FIN));
+      mbar_wait_bounded(bar(Cfg::BAR_FIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---- softmax warpgroups -----------------------------------------------------------
+    const int w = warp >> 2, r = threadIdx.x & (BM - 1);
+    const int qbase = qt * 2 * BM + w * BM;
+    const int nk = w == 0 ? nkt0 : nkt1;
+    if (qbase < n) {
+      // Q tile: row rr = query qbase + rr, zero past the new tokens
+      uint8_t* sQ = smem + Cfg::OFF_Q + w * Cfg::Q_BYTES;
+      constexpr int CH = D / 8;
+      for (int idx = r; idx < BM * CH; idx += BM) {
+        const int rr = idx / CH, c = idx % CH;
+        uint8_t* dst = sQ + (c >> 3) * (BM * 128) + sw128_off(rr, c & 7);
+        if (qbase + rr < n)
+          cp_async16(smem_addr(dst),
+                     static_cast<const T*>(a.q) + ((int64_t)(q0 + qbase + rr) * HQ + hq) * D + c * 8);
+        else
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_shared();
+      mbar_arrive(bar(Cfg::BAR_Q + w));
 
-  if (ok) {
-    // ---- O / l for this row -------------------------------------------------
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    T* dst = static_cast<T*>(a.out) + ((int64_t)(q0 + qi) * HQ + hq) * D;
+      const int qi = qbase + r;
+      const bool row_valid = qi < n;
+      const int pos = L - n + qi;  // this query's position
+      const float sl2 = a.scale_log2;
+      const float masked_raw = sl2 >= 0.f ? -INFINITY : INFINITY;
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t s_addr = tmem + lane_base + Cfg::S_COL0 + w * BN;
+      const uint32_t o_addr = tmem + lane_base + Cfg::O_COL0 + w * D;
+      uint8_t* sP = smem + Cfg::OFF_P + w * Cfg::NP * Cfg::P_BYTES;
+      float m_used = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nk; ++j) {
+        if (!(ok = warp_wait_or_abort(bar(Cfg::BAR_S + w), j & 1, abort_flag))) break;
+        tc_fence_after();
+        float sc[BN];
+        tmem_ld32_nowait(s_addr, sc);
+        tmem_ld32_nowait(s_addr + 32, sc + 32);
+        tmem_wait_ld();
+        const bool need_mask = !row_valid || j * BN + BN - 1 > pos;
+        if (need_mask) {
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      float o[32];
-      tmem_ld32(tmem + lane_base + Cfg::O_COL + c0, o);
-      if (row_valid) {
+          for (int c = 0; c < BN; ++c)
+            if (!row_valid || j * BN + c > pos) sc[c] = masked_raw;
+        }
+        // row max of the scaled scores (4 independent chains)
+        float mx4[4];
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
+        for (int i = 0; i < 4; ++i) mx4[i] = sc[i];
+        if (sl2 >= 0.f) {
+#pragma unroll
+          for (int c = 4; c < BN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], sc[c]);
+        } else {
+#pragma unroll
+          for (int c = 4; c < BN; ++c) mx4[c & 3] = fminf(mx4[c & 3], sc[c]);
+        }
+        const float mraw = sl2 >= 0.f ? fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]))
+                                      : fminf(fminf(mx4[0], mx4[1]), fminf(mx4[2], mx4[3]));
+        const float m_tile = sl2 == 0.f ? 0.f : mraw * sl2;
+        // move the reference max only when a weight would exceed 2^8
+        const bool move = m_tile > m_used + 8.f;
+        float alpha = 1.f;
+        if (move) {
+          alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+        }
+        const float mb = m_used == -INFINITY ? 0.f : m_used;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          sc[c] = ex2_approx(fmaf(sc[c], sl2, -mb));
+          sum4[c & 3] += sc[c];
+        }
+        if (need_mask) {  // a zero scale keeps masked scores finite: select them out
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (!row_valid || j * BN + c > pos) sc[c] = 0.f;
+          sum4[0] = sum4[1] = sum4[2] = sum4[3] = 0.f;
+#pragma unroll
+          for (int c = 0; c < BN; ++c) sum4[c & 3] += sc[c];
+        }
+        l_run = fmaf(l_run, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+        // rescale this row of O (P.V of tile j-1 has completed: the product
+        // S of tile j was committed after it)
+        __syncwarp();
+        if (j > 0 && __any_sync(kFullMask, move)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
+            tmem_ld32(o_addr + c0, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(o_addr + c0, o);
+          }
+        }
+        // this row of P into the swizzled A tile (64 keys = 8 chunks of 16 bytes)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
           uint4 v;
-          v.x = MmaType<T>::pack(o[i] * inv, o[i + 1] * inv);
-          v.y = MmaType<T>::pack(o[i + 2] * inv, o[i + 3] * inv);
-          v.z = MmaType<T>::pack(o[i + 4] * inv, o[i + 5] * inv);
-          v.w = MmaType<T>::pack(o[i + 6] * inv, o[i + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + c0 + i) = v;
+          if constexpr (Cfg::NP == 2) {
+            uint4 lo;
+            pack_split<T>(sc[8 * c + 0], sc[8 * c + 1], v.x, lo.x);
+            pack_split<T>(sc[8 * c + 2], sc[8 * c + 3], v.y, lo.y);
+            pack_split<T>(sc[8 * c + 4], sc[8 * c + 5], v.z, lo.z);
+            pack_split<T>(sc[8 * c + 6], sc[8 * c + 7], v.w, lo.w);
+            *reinterpret_cast<uint4*>(sP + Cfg::P_BYTES + sw128_off(r, c)) = lo;
+          } else {
+            v.x = MmaType<T>::pack(sc[8 * c + 0], sc[8 * c + 1]);
+            v.y = MmaType<T>::pack(sc[8 * c + 2], sc[8 * c + 3]);
+            v.z = MmaType<T>::pack(sc[8 * c + 4], sc[8 * c + 5]);
+            v.w = MmaType<T>::pack(sc[8 * c + 6], sc[8 * c + 7]);
+          }
+          *reinterpret_cast<uint4*>(sP + sw128_off(r, c)) = v;
+        }
+        fence_proxy_async_shared();
+        tc_fence_before();
+        mbar_arrive(bar(Cfg::BAR_P + w));
+      }
+      if (ok) ok = warp_wait_or_abort(bar(Cfg::BAR_O + w), 0, abort_flag);
+      if (!ok) {
+        give_up();
+      } else {
+        tc_fence_after();
+        // ---- O / l for this row -----------------------------------------------------
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        T* dst = static_cast<T*>(a.out) + ((int64_t)(q0 + qi) * HQ + hq) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float o[32];
+          tmem_ld32(o_addr + c0, o);
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = MmaType<T>::pack(o[i] * inv, o[i + 1] * inv);
+              v.y = MmaType<T>::pack(o[i + 2] * inv, o[i + 3] * inv);
+              v.z = MmaType<T>::pack(o[i + 4] * inv, o[i + 5] * inv);
+              v.w = MmaType<T>::pack(o[i + 6] * inv, o[i + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + c0 + i) = v;
+            }
+          }
         }
       }
     }
-  } else if (threadIdx.x == 0) {
-    atomicOr(a.err, PA_DEVERR_TIMEOUT);
   }
-  // let any copies still in flight land, then free TMEM
-  cp_async_wait<0>();
+  // every role is done and every copy or product it issued has landed
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

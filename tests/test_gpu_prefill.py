@@ -58,7 +58,8 @@ def _case(seed, ctx_new, kv_heads, group, head_dim, dtype):
     pool = pa.pa_pool_create(nb, 16, kv_heads, head_dim, tdt)
     pa.pa_pool_set_query_heads(pool, kv_heads * group)
     return dict(pool=pool, q=qt.cuda(), k=kt.cuda(), v=vt.cuda(), tables=dev(tables),
-                lens=dev(lens), qs=dev(qs), max_new=int(news.max()), ref=ref, scale=scale)
+                lens=dev(lens), qs=dev(qs), max_new=int(news.max()), ref=ref, scale=scale,
+                tables_h=tables)
 
 
 CASES = [(1, 1), (17, 17), (200, 64), (300, 300), (1000, 129), (128, 128), (2048, 256),
@@ -103,3 +104,29 @@ def test_prefill_rejects_a_context_shorter_than_its_new_tokens():
                             c["scale"], out, 20)
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
     assert_parity(out[:20], c["ref"][:20], "the valid sequence still runs")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_prefill_ignores_poisoned_rows_past_the_context(dtype):
+    """Pool rows past each context and blocks that no table holds are NaN: a
+    masked score and a zero weight must never meet them (0 x NaN in P.V)."""
+    ctx = [(45, 13), (300, 300), (17, 17), (1000, 129), (200, 64), (64, 64)]
+    c = _case(82, ctx, 2, 1, 128, dtype)
+    k, v = c["k"], c["v"]
+    used = np.zeros(k.shape[0], dtype=bool)
+    for s, (L, _) in enumerate(ctx):
+        nblk = math.ceil(L / 16)
+        blocks = c["tables_h"][s, :nblk]
+        used[blocks] = True
+        last, rows = int(blocks[-1]), L - (nblk - 1) * 16
+        k[last, :, rows:] = float("nan")
+        v[last, :, rows:] = float("nan")
+    free = torch.from_numpy(np.nonzero(~used)[0]).cuda()
+    k[free] = float("nan")
+    v[free] = float("nan")
+    out = torch.empty_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], k, v, c["tables"], c["lens"], c["qs"], c["scale"],
+                            out, c["max_new"])
+    assert pa.pa_device_errors() == 0
+    assert torch.isfinite(out.float()).all()
+    assert_parity(out, c["ref"], f"prefill {dtype} with NaN past the context")
