@@ -9,9 +9,10 @@
 // One CTA = (sequence, query head, 256 new queries as two 128-row tiles) with
 // specialised warps:
 //   * warps 0-3 and 4-7: two softmax warpgroups, one per query tile; thread r
-//     of a group owns query row r (TMEM lane r).  Each reads its row of S from
-//     TMEM, applies the causal mask and the online softmax in fp32 (log2
-//     domain) and writes its row of P (fp16/bf16) into a swizzled shared tile;
+//     of a group owns query row r (TMEM lane r).  Each reads its row of S
+//     (128 keys) from TMEM, applies the causal mask and the online softmax in
+//     fp32 (log2 domain) and writes its row of P (fp16/bf16 pairs) back over
+//     S in TMEM, where the P.V product takes its A operand from;
 //   * warp 8: the loader.  It streams the paged K and V rows of each 64-key
 //     tile with TMA tensor copies (one 16-row box per physical block and
 //     64-wide slice of head_dim, hardware 128-byte swizzle) into a ring of
@@ -21,11 +22,13 @@
 //     them to mbarriers.
 // The two query tiles share every K/V stage and take turns on the tensor core:
 // while one group runs its softmax, the MMA unit computes the other group's
-// P.V and next S.  The running max is only moved (and the row of O in TMEM
+// P.V and next S.  Keeping P in TMEM leaves shared memory to the Q, K and V
+// operands, whose bandwidth bounds the products (128-key tiles halve the Q
+// re-reads per flop against 64-key ones).  The running max is only moved (and the row of O in TMEM
 // rescaled) when a score exceeds it by more than 2^8, which keeps every
 // weight at most 256 and makes the rescale rare.
 // Shared-memory operands are described by SW128 matrix descriptors (K-major
-// for Q, K and P; MN-major for V).  Every wait is bounded; a wait that gives
+// for Q and K; MN-major for V).  Every wait is bounded; a wait that gives
 // up stops the CTA's other roles, lets every copy and product already issued
 // land, frees TMEM and reports PA_DEVERR_TIMEOUT.
 #pragma once
@@ -63,35 +66,45 @@ struct PrefillArgs {
 };
 
 // SPLIT_P: the softmax weights go to the tensor core as a high part plus its
-// rounding residual (two P tiles, two P.V chains).  bf16 needs it (8-bit
+// rounding residual (two P operands, two P.V chains).  bf16 needs it (8-bit
 // significand); fp16's 11 bits keep the result inside the parity gate alone.
 template <int D, bool SPLIT_P>
 struct PrefillConfig {
   static constexpr int BM = 128;        // query rows per tile (TMEM lanes)
   static constexpr int QT = 2;          // query tiles per CTA (softmax warpgroups)
-  static constexpr int BN = 64;         // keys per tile
+  static constexpr int BN = 128;        // keys per tile
   static constexpr int KB = D / 64;     // 128-byte K-blocks across head_dim
-  static constexpr int NS = 3;          // K/V ring stages
-  static constexpr int NP = SPLIT_P ? 2 : 1;
-  static constexpr int LOAD_WARP = 8, MMA_WARP = 9;
-  static constexpr int THREADS = 320;
+  static constexpr int NS = D == 128 ? 2 : 3;  // stages of the K ring and of the V ring
+  static constexpr int LOAD_WARP = 8, MMA_WARP = 9;  // warps 10-11 only fill the warpgroup
+  static constexpr int THREADS = 384;
+  // Launched at 168 registers a thread (384 x 168 fit the register file);
+  // the loader/MMA warpgroup then drops to 72 and the softmax groups rise to
+  // 216: 256 x 216 + 128 x 72 = 64512 = 384 x 168 launched (per SM
+  // sub-partition: two softmax warps and one other, 16128 of 16384).
+  static constexpr int REGS_LAUNCH = 168, REGS_SOFTMAX = 216, REGS_OTHER = 72;
+  static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * REGS_LAUNCH, "register split");
   static constexpr int Q_BYTES = KB * BM * 128;
-  static constexpr int KV_BYTES = KB * BN * 128;   // one of K or V
-  static constexpr int P_BYTES = BM * 128;         // BM rows x 64 keys
+  static constexpr int KV_BYTES = KB * BN * 128;   // one stage of K or of V
   static constexpr int OFF_Q = 0;                               // [tile]
-  static constexpr int OFF_KV = OFF_Q + QT * Q_BYTES;           // [stage][K|V]
-  static constexpr int OFF_P = OFF_KV + NS * 2 * KV_BYTES;      // [tile][high|residual]
-  static constexpr int OFF_BAR = OFF_P + QT * NP * P_BYTES;
-  // mbarriers: q_full[2], full[NS], empty[NS], s_full[2], p_full[2], o_done[2], fin
-  static constexpr int BAR_Q = 0, BAR_FULL = 2, BAR_EMPTY = 2 + NS, BAR_S = 2 + 2 * NS,
-                       BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_FIN = BAR_O + 2,
-                       NBARS = BAR_FIN + 1;
+  static constexpr int OFF_K = OFF_Q + QT * Q_BYTES;            // [stage]
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;           // [stage]
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  // mbarriers: q_full[2], K full/empty[NS], V full/empty[NS], s_full[2],
+  // p_full[2], o_done[2], fin
+  static constexpr int BAR_Q = 0, BAR_KF = 2, BAR_KE = BAR_KF + NS, BAR_VF = BAR_KE + NS,
+                       BAR_VE = BAR_VF + NS, BAR_S = BAR_VE + NS, BAR_P = BAR_S + 2,
+                       BAR_O = BAR_P + 2, BAR_FIN = BAR_O + 2, NBARS = BAR_FIN + 1;
   static constexpr int OFF_SLOT = OFF_BAR + NBARS * 8;  // TMEM address, abort flag
   // + 1 KB so the swizzled tiles can start on a 1024-byte boundary
   static constexpr size_t SMEM = OFF_SLOT + 16 + 1024;
-  static constexpr int S_COL0 = 0;                  // S of tile w at w * BN
-  static constexpr int O_COL0 = 2 * BN;             // O of tile w at O_COL0 + w * D
-  static constexpr int TMEM_COLS = (O_COL0 + 2 * D) <= 256 ? 256 : 512;
+  // TMEM columns: S of tile w at w * BN (fp32), overwritten by P as packed
+  // pairs (high part in its first 64 columns, residual in the next 64); O of
+  // tile w at O_COL0 + w * D.
+  static constexpr int S_COL0 = 0;
+  static constexpr int P_LO = 64;
+  static constexpr int O_COL0 = 2 * BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM columns");
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(SMEM <= 232448, "shared memory");
 };
@@ -122,6 +135,18 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same with A read from TMEM (rows on lanes, pairs of 16-bit elements
+// packed along K in each 32-bit column).
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -160,6 +185,19 @@ __device__ __forceinline__ void tmem_wait_ld() {
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   tmem_ld32_nowait(taddr, v);
   tmem_wait_ld();
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes from w (no wait).
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const uint32_t* w) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
@@ -220,6 +258,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+
 // Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile whose
 // rows are 128 bytes (one K-block).  The TMA copies with 128-byte swizzle
 // produce the same placement for boxes that start 1024-byte aligned.
@@ -233,7 +272,7 @@ constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
 // tm_k, tm_v: K and V pools viewed as [num_blocks * heads * 16 rows][head_dim],
 // box {64, 16} (one physical block, one 64-wide slice), 128-byte swizzle.
 template <typename T, int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     paged_prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -278,15 +317,17 @@ __global__ void __launch_bounds__(320, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (threadIdx.x == 32) {
-    mbar_init(bar(Cfg::BAR_Q + 0), BM);
-    mbar_init(bar(Cfg::BAR_Q + 1), BM);
+    mbar_init(bar(Cfg::BAR_Q + 0), BM / 32);  // one arrival per softmax warp
+    mbar_init(bar(Cfg::BAR_Q + 1), BM / 32);
     for (int i = 0; i < NS; ++i) {
-      mbar_init(bar(Cfg::BAR_FULL + i), 1);
-      mbar_init(bar(Cfg::BAR_EMPTY + i), 1);
+      mbar_init(bar(Cfg::BAR_KF + i), 1);
+      mbar_init(bar(Cfg::BAR_KE + i), 1);
+      mbar_init(bar(Cfg::BAR_VF + i), 1);
+      mbar_init(bar(Cfg::BAR_VE + i), 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Cfg::BAR_S + w), 1);
-      mbar_init(bar(Cfg::BAR_P + w), BM);
+      mbar_init(bar(Cfg::BAR_P + w), BM / 32);
       mbar_init(bar(Cfg::BAR_O + w), 1);
     }
     mbar_init(bar(Cfg::BAR_FIN), 1);
@@ -305,107 +346,143 @@ __global__ void __launch_bounds__(320, 1)
     }
   };
 
+  // registers move from the loader/MMA warpgroup to the softmax groups; each
+  // group changes its limit at one point, before its warps split into roles
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Cfg::REGS_OTHER));
   if (warp == Cfg::LOAD_WARP) {
-    // ---- loader: K and V of key tile j into stage j % NS ------------------------
+    // ---- loader: K and V of key tile j into stage j % NS of their rings ----------
+    // K runs one tile ahead of V: a K stage frees once both S products of its
+    // tile are issued, a V stage only after both P.V products.
     const int32_t* table = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-    int issued = 0;
-    for (int j = 0; j < nkt; ++j) {
-      const int st = j % NS;
-      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_EMPTY + st), ((j / NS) - 1) & 1, abort_flag)) {
-        give_up();
-        break;
-      }
-      const uint32_t sK = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES;
-      const uint32_t sV = sK + Cfg::KV_BYTES;
-      uint8_t* gV = smem + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES;
-      // V rows at or past the context are zeroed (their weights are zero, but
-      // stale bits may be NaN); K rows there are masked out of S by selection.
-      // A partly filled last block's valid V rows are copied by the lanes, so
-      // every tensor copy moves a whole block.
-      const int valid_in_tile = min(BN, L - j * BN);
-      const int nblk = (valid_in_tile + kBlock - 1) / kBlock;  // blocks holding tokens
-      const bool partial = valid_in_tile < nblk * kBlock;
-      auto block_of = [&](int i) {
-        int32_t blk = table[j * (BN / kBlock) + i];
+    int k_issued = 0, v_issued = 0;
+    // lane i < blocks in tile j: that block's id (fetched by all lanes at once)
+    auto tile_blocks = [&](int j, int& nblk, int& valid) {
+      valid = min(BN, L - j * BN);
+      nblk = (valid + kBlock - 1) / kBlock;
+      int32_t blk = 0;
+      if (lane < nblk) {
+        blk = table[j * (BN / kBlock) + lane];
         if (blk < 0 || blk >= a.num_blocks) {
           atomicOr(a.err, PA_DEVERR_BLOCK_ID);
           blk = 0;
         }
-        return blk;
-      };
-      if (valid_in_tile < BN) {
-        const int r_lo = partial ? (nblk - 1) * kBlock : valid_in_tile;
-        const T* src = nullptr;
-        if (partial)
-          src = static_cast<const T*>(a.v_pool) +
-                (((int64_t)block_of(nblk - 1) * a.heads + kvh) * kBlock) * D;
+      }
+      return blk;
+    };
+    auto load_k = [&](int j) {
+      int nblk, valid;
+      const int32_t blk = tile_blocks(j, nblk, valid);
+      const int st = j % NS;
+      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_KE + st), ((j / NS) - 1) & 1, abort_flag))
+        return false;
+      if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_KF + st), (uint32_t)nblk * KB * kBlock * 128);
+      __syncwarp();
+      if (lane < nblk) {  // K rows past the context are masked out of S by selection
+        const int row0 = (int)(((int64_t)blk * a.heads + kvh) * kBlock);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(sbase + Cfg::OFF_K + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
+                      &tm_k, kb * 64, row0, bar(Cfg::BAR_KF + st));
+      }
+      k_issued = j + 1;
+      return true;
+    };
+    auto load_v = [&](int j) {
+      int nblk, valid;
+      const int32_t blk = tile_blocks(j, nblk, valid);
+      const int st = j % NS;
+      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_VE + st), ((j / NS) - 1) & 1, abort_flag))
+        return false;
+      // V rows at or past the context are zeroed (their weights are zero, but
+      // stale bits may be NaN).  A partly filled last block's valid rows are
+      // copied by the lanes, so every tensor copy moves a whole block.
+      const bool partial = valid < nblk * kBlock;
+      const int32_t last_blk = __shfl_sync(kFullMask, blk, nblk - 1);
+      uint8_t* gV = smem + Cfg::OFF_V + st * Cfg::KV_BYTES;
+      if (valid < BN) {
+        const int r_lo = partial ? (nblk - 1) * kBlock : valid;
+        const T* src = static_cast<const T*>(a.v_pool) +
+                       (((int64_t)last_blk * a.heads + kvh) * kBlock) * D;
         for (int idx = lane; idx < (BN - r_lo) * KB * 8; idx += 32) {
           const int r = r_lo + idx / (KB * 8), c = idx % (KB * 8);
           uint4 v = make_uint4(0, 0, 0, 0);
-          if (r < valid_in_tile)
-            v = *reinterpret_cast<const uint4*>(src + (int64_t)(r - r_lo) * D + c * 8);
+          if (r < valid) v = *reinterpret_cast<const uint4*>(src + (int64_t)(r - r_lo) * D + c * 8);
           *reinterpret_cast<uint4*>(gV + (c >> 3) * (BN * 128) + sw128_off(r, c & 7)) = v;
         }
         fence_proxy_async_shared();
       }
+      const int nfull = partial ? nblk - 1 : nblk;
       __syncwarp();
-      if (lane == 0) {
-        const int nfull_v = partial ? nblk - 1 : nblk;
-        const uint32_t bytes = (uint32_t)(nblk + nfull_v) * KB * kBlock * 128;
-        mbar_arrive_expect_tx(bar(Cfg::BAR_FULL + st), bytes);
-        for (int i = 0; i < nblk; ++i) {
-          const int row0 = (int)(((int64_t)block_of(i) * a.heads + kvh) * kBlock);
+      if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_VF + st), (uint32_t)nfull * KB * kBlock * 128);
+      __syncwarp();
+      if (lane < nfull) {
+        const int row0 = (int)(((int64_t)blk * a.heads + kvh) * kBlock);
 #pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            const uint32_t o = kb * (BN * 128) + i * (kBlock * 128);
-            tma_load_2d(sK + o, &tm_k, kb * 64, row0, bar(Cfg::BAR_FULL + st));
-            if (i < nfull_v) tma_load_2d(sV + o, &tm_v, kb * 64, row0, bar(Cfg::BAR_FULL + st));
-          }
-        }
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(sbase + Cfg::OFF_V + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
+                      &tm_v, kb * 64, row0, bar(Cfg::BAR_VF + st));
       }
-      issued = j + 1;
+      v_issued = j + 1;
+      return true;
+    };
+    for (int t = 0; t <= nkt; ++t) {
+      if ((t < nkt && !load_k(t)) || (t >= 1 && !load_v(t - 1))) {
+        give_up();
+        break;
+      }
     }
     // let the copies of the last stages land before the CTA releases its memory
-    if (lane == 0)
-      for (int j = max(0, issued - NS); j < issued; ++j)
-        mbar_wait_bounded(bar(Cfg::BAR_FULL + j % NS), (j / NS) & 1);
+    if (lane == 0) {
+      for (int j = max(0, k_issued - NS); j < k_issued; ++j)
+        mbar_wait_bounded(bar(Cfg::BAR_KF + j % NS), (j / NS) & 1);
+      for (int j = max(0, v_issued - NS); j < v_issued; ++j)
+        mbar_wait_bounded(bar(Cfg::BAR_VF + j % NS), (j / NS) & 1);
+    }
   } else if (warp == Cfg::MMA_WARP) {
     // ---- MMA issue ------------------------------------------------------------------
     if (lane == 0) {
+      // Descriptors are built once: an operand at a byte offset o from a
+      // base differs only in the start-address field (o >> 4 added to the
+      // low word; every address here stays inside that 14-bit field), so a
+      // product costs one add per operand on the issuing thread, which
+      // shares its sub-partition with two busy softmax warps.
+      const uint64_t dq = sw128_desc(sbase + Cfg::OFF_Q, 16, 1024);
+      const uint64_t dk = sw128_desc(sbase + Cfg::OFF_K, 16, 1024);
+      const uint64_t dv = sw128_desc(sbase + Cfg::OFF_V, BN * 128, 1024);
+      auto at = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
       auto issue_s = [&](int w, int st) {
-        const uint32_t qa = sbase + Cfg::OFF_Q + w * Cfg::Q_BYTES;
-        const uint32_t ka = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES;
+        const uint64_t qd = at(dq, w * Cfg::Q_BYTES), kd = at(dk, st * Cfg::KV_BYTES);
+        const uint32_t sd = tmem + Cfg::S_COL0 + w * BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t kofs = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
           const uint32_t kofs_b = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          umma_f16(tmem + Cfg::S_COL0 + w * BN, sw128_desc(qa + kofs, 16, 1024),
-                   sw128_desc(ka + kofs_b, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          umma_f16(sd, at(qd, kofs), at(kd, kofs_b), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int w, int st, bool first) {
-        const uint32_t pa = sbase + Cfg::OFF_P + w * Cfg::NP * Cfg::P_BYTES;
-        const uint32_t va = sbase + Cfg::OFF_KV + st * 2 * Cfg::KV_BYTES + Cfg::KV_BYTES;
+        const uint32_t pa = tmem + Cfg::S_COL0 + w * BN;  // P over S, 8 columns per 16 keys
+        const uint32_t od = tmem + Cfg::O_COL0 + w * D;
+        const uint64_t vd = at(dv, st * Cfg::KV_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // V is MN-major: 64-dim blocks LBO apart, 8-key groups 1024 bytes apart
-          const uint64_t bd = sw128_desc(va + kk * 2048, BN * 128, 1024);
-          umma_f16(tmem + Cfg::O_COL0 + w * D, sw128_desc(pa + kk * 32, 16, 1024), bd, IDESC_PV,
-                   (!first || kk > 0) ? 1u : 0u);
-          if constexpr (Cfg::NP == 2)
-            umma_f16(tmem + Cfg::O_COL0 + w * D,
-                     sw128_desc(pa + Cfg::P_BYTES + kk * 32, 16, 1024), bd, IDESC_PV, 1u);
+          const uint64_t bd = at(vd, kk * 2048);
+          umma_f16_ts(od, pa + kk * 8, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          if constexpr (kSplitP<T>) umma_f16_ts(od, pa + Cfg::P_LO + kk * 8, bd, IDESC_PV, 1u);
         }
       };
-      int ready = -1;  // last key tile whose stage was seen full
-      auto wait_kv = [&](int j) {
+      int k_ready = -1, v_ready = -1;  // last tiles whose K / V stage was seen full
+      auto wait_full = [&](int base, int j, int& ready) {
         if (j <= ready) return true;
-        if (!mbar_wait_or_abort(bar(Cfg::BAR_FULL + j % NS), (j / NS) & 1, abort_flag)) return false;
+        if (!mbar_wait_or_abort(bar(base + j % NS), (j / NS) & 1, abort_flag)) return false;
         ready = j;
         tc_fence_after();
         return true;
       };
-      bool ok = mbar_wait_or_abort(bar(Cfg::BAR_Q + 0), 0, abort_flag) && wait_kv(0) &&
+      bool ok = mbar_wait_or_abort(bar(Cfg::BAR_Q + 0), 0, abort_flag) &&
+                wait_full(Cfg::BAR_KF, 0, k_ready) &&
                 (!has1 || mbar_wait_or_abort(bar(Cfg::BAR_Q + 1), 0, abort_flag));
       if (ok) {
         tc_fence_after();
@@ -415,25 +492,30 @@ __global__ void __launch_bounds__(320, 1)
           issue_s(1, 0);
           umma_commit(bar(Cfg::BAR_S + 1));
         }
+        umma_commit(bar(Cfg::BAR_KE + 0));
       }
       for (int j = 0; ok && j < nkt; ++j) {
-        const int st = j % NS;
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const int nk = w == 0 ? nkt0 : nkt1;
           if (j >= nk) continue;
-          if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + w), j & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + w), j & 1, abort_flag) &&
+                     wait_full(Cfg::BAR_VF, j, v_ready)))
+            break;
           tc_fence_after();
-          issue_pv(w, st, j == 0);
+          issue_pv(w, j % NS, j == 0);
           if (j == nk - 1) {
             umma_commit(bar(Cfg::BAR_O + w));
           } else {
-            if (!(ok = wait_kv(j + 1))) break;
+            if (!(ok = wait_full(Cfg::BAR_KF, j + 1, k_ready))) break;
             issue_s(w, (j + 1) % NS);
             umma_commit(bar(Cfg::BAR_S + w));
           }
         }
-        if (ok) umma_commit(bar(Cfg::BAR_EMPTY + st));
+        if (ok) {
+          umma_commit(bar(Cfg::BAR_VE + j % NS));
+          if (j + 1 < nkt) umma_commit(bar(Cfg::BAR_KE + (j + 1) % NS));
+        }
       }
       if (!ok) give_up();
       // every product issued has completed before TMEM and shared memory go
@@ -441,7 +523,9 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait_bounded(bar(Cfg::BAR_FIN), 0);
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Cfg::REGS_SOFTMAX));
     // ---- softmax warpgroups -----------------------------------------------------------
     const int w = warp >> 2, r = threadIdx.x & (BM - 1);
     const int qbase = qt * 2 * BM + w * BM;
@@ -462,7 +546,8 @@ __global__ void __launch_bounds__(320, 1)
       cp_async_commit();
       cp_async_wait<0>();
       fence_proxy_async_shared();
-      mbar_arrive(bar(Cfg::BAR_Q + w));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Cfg::BAR_Q + w));
 
       const int qi = qbase + r;
       const bool row_valid = qi < n;
@@ -472,15 +557,15 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t s_addr = tmem + lane_base + Cfg::S_COL0 + w * BN;
       const uint32_t o_addr = tmem + lane_base + Cfg::O_COL0 + w * D;
-      uint8_t* sP = smem + Cfg::OFF_P + w * Cfg::NP * Cfg::P_BYTES;
       float m_used = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < nk; ++j) {
         if (!(ok = warp_wait_or_abort(bar(Cfg::BAR_S + w), j & 1, abort_flag))) break;
         tc_fence_after();
-        float sc[BN];
-        tmem_ld32_nowait(s_addr, sc);
-        tmem_ld32_nowait(s_addr + 32, sc + 32);
+        float2 sv[BN / 2];
+        float* sc = reinterpret_cast<float*>(sv);
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) tmem_ld32_nowait(s_addr + c0, sc + c0);
         tmem_wait_ld();
         const bool need_mask = !row_valid || j * BN + BN - 1 > pos;
         if (need_mask) {
@@ -488,19 +573,26 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < BN; ++c)
             if (!row_valid || j * BN + c > pos) sc[c] = masked_raw;
         }
-        // row max of the scaled scores (4 independent chains)
-        float mx4[4];
+        // row max of the scaled scores (8 independent chains)
+        float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mx4[i] = sc[i];
+        for (int i = 0; i < 8; ++i) mx8[i] = sc[i];
         if (sl2 >= 0.f) {
 #pragma unroll
-          for (int c = 4; c < BN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], sc[c]);
+          for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sc[c]);
+#pragma unroll
+          for (int i = 4; i >= 1; i >>= 1)
+#pragma unroll
+            for (int k = 0; k < i; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + i]);
         } else {
 #pragma unroll
-          for (int c = 4; c < BN; ++c) mx4[c & 3] = fminf(mx4[c & 3], sc[c]);
+          for (int c = 8; c < BN; ++c) mx8[c & 7] = fminf(mx8[c & 7], sc[c]);
+#pragma unroll
+          for (int i = 4; i >= 1; i >>= 1)
+#pragma unroll
+            for (int k = 0; k < i; ++k) mx8[k] = fminf(mx8[k], mx8[k + i]);
         }
-        const float mraw = sl2 >= 0.f ? fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]))
-                                      : fminf(fminf(mx4[0], mx4[1]), fminf(mx4[2], mx4[3]));
+        const float mraw = mx8[0];
         const float m_tile = sl2 == 0.f ? 0.f : mraw * sl2;
         // move the reference max only when a weight would exceed 2^8
         const bool move = m_tile > m_used + 8.f;
@@ -510,21 +602,26 @@ __global__ void __launch_bounds__(320, 1)
           m_used = m_tile;
         }
         const float mb = m_used == -INFINITY ? 0.f : m_used;
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 sl2v = make_float2(sl2, sl2), nmb = make_float2(-mb, -mb);
+        // weights in fp32: exp2 on the multi-function unit (4 per clock per
+        // sub-partition, in step with the tensor core's work on the tile)
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          sc[c] = ex2_approx(fmaf(sc[c], sl2, -mb));
-          sum4[c & 3] += sc[c];
+        for (int i = 0; i < BN / 2; ++i) {
+          const float2 x = __ffma2_rn(sv[i], sl2v, nmb);
+          sv[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
         }
         if (need_mask) {  // a zero scale keeps masked scores finite: select them out
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (!row_valid || j * BN + c > pos) sc[c] = 0.f;
-          sum4[0] = sum4[1] = sum4[2] = sum4[3] = 0.f;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) sum4[c & 3] += sc[c];
         }
-        l_run = fmaf(l_run, alpha, (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+        float2 sum4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum4[i] = sv[i];
+#pragma unroll
+        for (int i = 4; i < BN / 2; ++i) sum4[i & 3] = __fadd2_rn(sum4[i & 3], sv[i]);
+        sum4[0] = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
+        l_run = fmaf(l_run, alpha, sum4[0].x + sum4[0].y);
         // rescale this row of O (P.V of tile j-1 has completed: the product
         // S of tile j was committed after it)
         __syncwarp();
@@ -538,28 +635,29 @@ __global__ void __launch_bounds__(320, 1)
             tmem_st32(o_addr + c0, o);
           }
         }
-        // this row of P into the swizzled A tile (64 keys = 8 chunks of 16 bytes)
+        // this row of P over S in TMEM: column c holds keys 2c (low half) and
+        // 2c + 1; the S values were all read above
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v;
-          if constexpr (Cfg::NP == 2) {
-            uint4 lo;
-            pack_split<T>(sc[8 * c + 0], sc[8 * c + 1], v.x, lo.x);
-            pack_split<T>(sc[8 * c + 2], sc[8 * c + 3], v.y, lo.y);
-            pack_split<T>(sc[8 * c + 4], sc[8 * c + 5], v.z, lo.z);
-            pack_split<T>(sc[8 * c + 6], sc[8 * c + 7], v.w, lo.w);
-            *reinterpret_cast<uint4*>(sP + Cfg::P_BYTES + sw128_off(r, c)) = lo;
+        for (int h = 0; h < BN / 32; ++h) {
+          if constexpr (kSplitP<T>) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pack_split<T>(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1], hi[i], lo[i]);
+            tmem_st16_nowait(s_addr + Cfg::P_LO + 16 * h, lo);
+            tmem_st16_nowait(s_addr + 16 * h, hi);
           } else {
-            v.x = MmaType<T>::pack(sc[8 * c + 0], sc[8 * c + 1]);
-            v.y = MmaType<T>::pack(sc[8 * c + 2], sc[8 * c + 3]);
-            v.z = MmaType<T>::pack(sc[8 * c + 4], sc[8 * c + 5]);
-            v.w = MmaType<T>::pack(sc[8 * c + 6], sc[8 * c + 7]);
+            uint32_t hi[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              hi[i] = MmaType<T>::pack(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1]);
+            tmem_st16_nowait(s_addr + 16 * h, hi);
           }
-          *reinterpret_cast<uint4*>(sP + sw128_off(r, c)) = v;
         }
-        fence_proxy_async_shared();
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(Cfg::BAR_P + w));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(Cfg::BAR_P + w));
       }
       if (ok) ok = warp_wait_or_abort(bar(Cfg::BAR_O + w), 0, abort_flag);
       if (!ok) {
