@@ -1,0 +1,218 @@
+"""Per-kernel timings on synthetic workloads (CUDA events on the launching stream).
+
+    python -m paged_kv_cache_478_b200.kernel_bench prefill [--small]
+    python -m paged_kv_cache_478_b200.kernel_bench gqa
+    python -m paged_kv_cache_478_b200.kernel_bench shared-prefix
+    python -m paged_kv_cache_478_b200.kernel_bench long-context
+
+Each line printed is one JSON object.  These are the measurements behind the
+per-kernel tables of the design notes; the headline decode step is bench.py.
+`prefill --small` runs three launches of one small case (2 prompts x 2048
+tokens) and prints nothing timed: it is the command the profiler captures.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+
+import numpy as np
+import torch
+
+import paged_kv_cache_478_b200 as pa
+from paged_kv_cache_478_b200 import synthetic as syn
+
+
+def _events_ms(fn, reps: int, warmup: int = 3, flush: torch.Tensor | None = None) -> float:
+    """Median milliseconds of fn() over reps, each bracketed by events on the
+    current stream; with `flush`, L2 is overwritten before every rep."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
+
+
+def _check():
+    err = pa.pa_device_errors()
+    if err:
+        raise RuntimeError(f"device error bits 0x{err:x}")
+
+
+def _prefill_case(seqs, new_tokens, kv_heads, group, head_dim, dtype, seed=0):
+    lens = np.full(seqs, new_tokens, dtype=np.int32)
+    need = math.ceil(new_tokens / 16)
+    nb = seqs * need
+    tables = np.random.default_rng(seed).permutation(nb).astype(np.int32).reshape(seqs, need)
+    kp = torch.empty((nb, kv_heads, 16, head_dim), dtype=dtype, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 1)
+    syn.fill_normal_device(vp, 2)
+    q = torch.empty((seqs * new_tokens, kv_heads * group, head_dim), dtype=dtype, device="cuda")
+    syn.fill_normal_device(q, 3)
+    qs = torch.arange(0, seqs * new_tokens + 1, new_tokens, dtype=torch.int32, device="cuda")
+    pool = pa.pa_pool_create(nb, 16, kv_heads, head_dim, dtype)
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    out = torch.empty_like(q)
+    scale = 1 / math.sqrt(head_dim)
+
+    def run():
+        pa.pa_prefill_attention(pool, q, kp, vp, bt, cl, qs, scale, out, new_tokens)
+
+    # causal attention of fresh prompts: Q.K^T and P.V over the lower triangle
+    flops = 4.0 * seqs * kv_heads * group * head_dim * new_tokens * (new_tokens + 1) / 2
+    return run, flops
+
+
+def prefill(small: bool):
+    if small:
+        run, _ = _prefill_case(2, 2048, 32, 1, 128, torch.float16)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        _check()
+        print(json.dumps({"prefill_small_case": "2 x 2048 fp16, 32 heads x 128, 3 launches"}))
+        return
+    for seqs, n, hk, g, dt in [(4, 4096, 32, 1, torch.float16), (8, 2048, 32, 1, torch.float16),
+                               (16, 1024, 8, 4, torch.float16), (8, 2048, 32, 1, torch.bfloat16)]:
+        run, flops = _prefill_case(seqs, n, hk, g, 128, dt)
+        ms = _events_ms(run, 20)
+        _check()
+        print(json.dumps({"kernel": "paged_prefill_kernel", "prompts": seqs, "new_tokens": n,
+                          "q_heads": hk * g, "kv_heads": hk, "dtype": str(dt).split(".")[-1],
+                          "ms": round(ms, 4), "TFLOPs": round(flops / ms / 1e9, 1)}), flush=True)
+
+
+def gqa():
+    S, HK, D = 200, 8, 128
+    lens = syn.full_step_lengths(0, S)
+    tables, nb = syn.full_step_tables(0, lens)
+    kp = torch.empty((nb, HK, 16, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 1)
+    syn.fill_normal_device(vp, 2)
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    kv_bytes = int(lens.sum()) * HK * D * 2 * 2
+    for G in (1, 2, 4, 8):
+        pool = pa.pa_pool_create(nb, 16, HK, D, torch.float16)
+        pa.pa_pool_set_query_heads(pool, HK * G)
+        q = torch.randn((S, HK * G, D), dtype=torch.float16, device="cuda")
+        kn = torch.randn((S, HK, D), dtype=torch.float16, device="cuda")
+        vn = torch.randn_like(kn)
+        out = torch.empty_like(q)
+        ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
+                         device="cuda")
+        pa.pa_decode_plan(pool, cl, tables.shape[1], ws)
+        ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
+            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws), 50)
+        _check()
+        print(json.dumps({"kernel": "decode (GQA)", "q_per_kv": G, "kv_heads": HK,
+                          "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}),
+              flush=True)
+
+
+def shared_prefix():
+    H, D, S, P = 32, 128, 128, 1000
+    case = syn.shared_prefix_case(0)
+    nb = 63 + S + sum(math.ceil(int(n) / 16) for n in case["suffix_lens"])
+    bm = pa.BlockManager(nb)
+    maxb = math.ceil((P + 512) / 16)
+    tables = np.full((S, maxb), -1, dtype=np.int32)
+    lens = np.zeros(S, dtype=np.int32)
+    lens[0], _, _ = bm.append_tokens(tables[0], 0, P)
+    for s in range(1, S):
+        bm.fork_table(tables[0], 63, tables[s])
+        lens[s] = P
+    for s in range(S):
+        lens[s], _, _ = bm.append_tokens(tables[s], int(lens[s]), int(case["suffix_lens"][s]))
+    kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 3)
+    syn.fill_normal_device(vp, 4)
+    pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
+    q = torch.randn((S, H, D), dtype=torch.float16, device="cuda")
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    groups = pa.pa_find_shared_prefixes(tables, lens)
+    gd = dict(groups)
+    for k in ("offsets", "members", "blocks"):
+        gd[k] = torch.from_numpy(groups[k]).cuda()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    used = {int(b) for s in range(S) for b in tables[s, :math.ceil(int(lens[s]) / 16)]}
+    unique = len(used) * H * 16 * D * 2 * 2
+    logical = int(lens.sum()) * H * D * 2 * 2
+    out1, out2 = torch.empty_like(q), torch.empty_like(q)
+    ws1 = torch.empty(pa.pa_decode_workspace_bytes(pool, S, maxb), dtype=torch.uint8, device="cuda")
+    ws2 = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(pool, S, maxb,
+                                                                  groups["max_shared_blocks"]),
+                      dtype=torch.uint8, device="cuda")
+    scale = 1 / math.sqrt(D)
+    t1 = _events_ms(lambda: pa.pa_decode_attention(pool, q, kp, vp, bt, cl, scale, out1, ws1), 50,
+                    flush=flush)
+    t2 = _events_ms(lambda: pa.pa_decode_attention_shared_prefix(pool, q, kp, vp, bt, cl, gd, scale,
+                                                                 out2, ws2), 50, flush=flush)
+    _check()
+    diff = (out1.float() - out2.float()).abs().max().item()
+    for name, ms in (("plain decode", t1), ("shared-prefix path", t2)):
+        print(json.dumps({"kernel": name, "sequences": S, "shared_prefix_tokens": P,
+                          "us": round(ms * 1e3, 1), "logical_GBps": round(logical / ms / 1e6, 1),
+                          "unique_GBps": round(unique / ms / 1e6, 1),
+                          "max_abs_diff_vs_plain": diff, "l2": "flushed before every rep"}),
+              flush=True)
+
+
+def long_context():
+    S, H, D, CTX = 8, 32, 128, 32768
+    lens, tables, nb = syn.long_context_tables(0, S, CTX)
+    kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 1)
+    syn.fill_normal_device(vp, 2)
+    q = torch.randn((S, H, D), dtype=torch.float16, device="cuda")
+    kn, vn = torch.randn_like(q), torch.randn_like(q)
+    pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty_like(q)
+    pa.pa_decode_plan(pool, cl, tables.shape[1], ws)
+    ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
+        pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws), 30)
+    _check()
+    kv_bytes = int(lens.sum()) * H * D * 2 * 2
+    print(json.dumps({"kernel": "decode (long context)", "sequences": S, "context": CTX,
+                      "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    sub = ap.add_subparsers(dest="what", required=True)
+    p = sub.add_parser("prefill")
+    p.add_argument("--small", action="store_true", help="3 launches of 2 x 2048 fp16 (profiling)")
+    sub.add_parser("gqa")
+    sub.add_parser("shared-prefix")
+    sub.add_parser("long-context")
+    args = ap.parse_args(argv)
+    if not torch.cuda.is_available():
+        raise SystemExit("kernel_bench needs a CUDA device")
+    if args.what == "prefill":
+        prefill(args.small)
+    elif args.what == "gqa":
+        gqa()
+    elif args.what == "shared-prefix":
+        shared_prefix()
+    else:
+        long_context()
+
+
+if __name__ == "__main__":
+    main()
