@@ -24,12 +24,14 @@ from paged_kv_cache_478_b200 import synthetic as syn
 
 
 def _events_ms(fn, reps: int, warmup: int = 3, flush: torch.Tensor | None = None) -> float:
-    """Median milliseconds of fn() over reps, each bracketed by events on the
-    current stream; with `flush`, L2 is overwritten before every rep."""
+    """Median milliseconds of fn() over reps, each bracketed by its own pair of
+    events on the current stream; with `flush`, L2 is overwritten before every
+    rep (outside the events).  All reps are queued before one synchronise, so
+    the device never waits on the host between an event pair."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    times = []
+    pairs = []
     for _ in range(reps):
         if flush is not None:
             flush.zero_()
@@ -37,9 +39,9 @@ def _events_ms(fn, reps: int, warmup: int = 3, flush: torch.Tensor | None = None
         e0.record()
         fn()
         e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-    return float(np.median(times))
+        pairs.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.median([e0.elapsed_time(e1) for e0, e1 in pairs]))
 
 
 def _check():
