@@ -5,8 +5,11 @@
 // a [G x 16] . [16 x D] value product, i.e. two m16n8k16 chains with the G
 // query heads as the rows.  One warp owns one KV head of the work item and
 // all of its query heads, so the CUDA-core cost per byte no longer grows
-// with G.  The softmax weights enter P.V as a high part plus its rounding
-// residual, so bf16 operands do not cost the result precision.  The pipeline
+// with G.  With bf16 the softmax weights enter P.V as a high part plus its
+// rounding residual (8 significand bits alone would cost the result
+// precision); fp16 weights go in as they are.  The running max only moves,
+// and the accumulators are only rescaled, when a score passes it by more than
+// 2^8, so the rescale is rare and the weights stay at most 256.  The pipeline
 // is the MHA kernel's: a per-warp NSTAGE ring fed by
 // 1-D bulk copies on mbarriers, items from the plan's queue, split-K partials
 // merged by the last CTA to finish a sequence, optional fused append.  Rows
@@ -18,6 +21,8 @@
 
 #include <math.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "decode.cuh"
 #include "device_utils.cuh"
@@ -209,23 +214,37 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
         float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
         mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = exp2f(m_run - m_new);
-        const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
-        const float p2 = exp2f(x2 - m_new), p3 = exp2f(x3 - m_new);
+        // the reference max moves only when a weight would pass 2^8 (the four
+        // lanes of a query row agree: mx is their common maximum)
+        const bool move = mx > m_run + 8.f;
+        float alpha = 1.f;
+        if (move) {
+          alpha = exp2f(m_run - mx);  // 0 on the first move
+          m_run = mx;
+        }
+        const float mb = m_run == -INFINITY ? 0.f : m_run;
+        const float p0 = exp2f(x0 - mb), p1 = exp2f(x1 - mb);
+        const float p2 = exp2f(x2 - mb), p3 = exp2f(x3 - mb);
         float sum = (p0 + p1) + (p2 + p3);
         sum += __shfl_xor_sync(kFullMask, sum, 1);
         sum += __shfl_xor_sync(kFullMask, sum, 2);
         l_run = fmaf(l_run, alpha, sum);
-        m_run = m_new;
+        if (__any_sync(kFullMask, move)) {
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          o[j][0] *= alpha;
-          o[j][1] *= alpha;
+          for (int j = 0; j < NT; ++j) {
+            o[j][0] *= alpha;
+            o[j][1] *= alpha;
+          }
         }
+        constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
         uint32_t pa_[4] = {0u, 0u, 0u, 0u}, pl_[4] = {0u, 0u, 0u, 0u};
-        pack_split<T>(p0, p1, pa_[0], pl_[0]);
-        pack_split<T>(p2, p3, pa_[2], pl_[2]);
+        if constexpr (kSplit) {
+          pack_split<T>(p0, p1, pa_[0], pl_[0]);
+          pack_split<T>(p2, p3, pa_[2], pl_[2]);
+        } else {
+          pa_[0] = MmaType<T>::pack(p0, p1);
+          pa_[2] = MmaType<T>::pack(p2, p3);
+        }
         {
           const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
           const int col = (lane >> 4) * 8;
@@ -236,9 +255,11 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
             float d0[4] = {o[j][0], o[j][1], 0.f, 0.f};
             float d1[4] = {o[j + 1][0], o[j + 1][1], 0.f, 0.f};
             mma16816<T>(d0, pa_, b[0], b[1]);
-            mma16816<T>(d0, pl_, b[0], b[1]);
             mma16816<T>(d1, pa_, b[2], b[3]);
-            mma16816<T>(d1, pl_, b[2], b[3]);
+            if constexpr (kSplit) {
+              mma16816<T>(d0, pl_, b[0], b[1]);
+              mma16816<T>(d1, pl_, b[2], b[3]);
+            }
             o[j][0] = d0[0];
             o[j][1] = d0[1];
             o[j + 1][0] = d1[0];

@@ -296,8 +296,11 @@ int auto_partition(int num_seqs, int head_groups, int max_context_len, int slots
   const int64_t whole = (int64_t)num_seqs * head_groups;
   const int64_t maxL = std::max(16, max_context_len);
   if (whole >= 2LL * slots) return std::min(kFullBatchPartition, round_up16(maxL));
+  // About 4 work items per resident CTA.  Only the longest context is known
+  // here; a ragged batch averages about half of it, so the partitions are
+  // sized for maxL / 2 (sizing them for maxL left items too long to balance).
   const int64_t want_parts = (4LL * slots + whole - 1) / std::max<int64_t>(whole, 1);
-  const int64_t ps = (maxL + want_parts - 1) / want_parts;
+  const int64_t ps = (maxL / 2 + want_parts - 1) / want_parts;
   return std::max(kMinAutoPartition, round_up16(ps));
 }
 

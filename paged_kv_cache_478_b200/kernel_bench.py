@@ -95,7 +95,7 @@ def prefill(small: bool):
                           "ms": round(ms, 4), "TFLOPs": round(flops / ms / 1e9, 1)}), flush=True)
 
 
-def gqa():
+def gqa(partition_size: int = 0):
     S, HK, D = 200, 8, 128
     lens = syn.full_step_lengths(0, S)
     tables, nb = syn.full_step_tables(0, lens)
@@ -112,13 +112,15 @@ def gqa():
         kn = torch.randn((S, HK, D), dtype=torch.float16, device="cuda")
         vn = torch.randn_like(kn)
         out = torch.empty_like(q)
-        ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
-                         device="cuda")
-        pa.pa_decode_plan(pool, cl, tables.shape[1], ws)
+        ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, partition_size),
+                         dtype=torch.uint8, device="cuda")
+        pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=partition_size)
         ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
-            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws), 50)
+            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size),
+            50)
         _check()
         print(json.dumps({"kernel": "decode (GQA)", "q_per_kv": G, "kv_heads": HK,
+                          "partition_size": partition_size or "auto",
                           "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}),
               flush=True)
 
@@ -172,7 +174,7 @@ def shared_prefix():
               flush=True)
 
 
-def long_context():
+def long_context(partition_size: int = 0):
     S, H, D, CTX = 8, 32, 128, 32768
     lens, tables, nb = syn.long_context_tables(0, S, CTX)
     kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
@@ -183,15 +185,16 @@ def long_context():
     kn, vn = torch.randn_like(q), torch.randn_like(q)
     pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
     bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
-    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, partition_size),
+                     dtype=torch.uint8, device="cuda")
     out = torch.empty_like(q)
-    pa.pa_decode_plan(pool, cl, tables.shape[1], ws)
+    pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=partition_size)
     ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
-        pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws), 30)
+        pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size), 30)
     _check()
     kv_bytes = int(lens.sum()) * H * D * 2 * 2
     print(json.dumps({"kernel": "decode (long context)", "sequences": S, "context": CTX,
+                      "partition_size": partition_size or "auto",
                       "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
@@ -200,20 +203,22 @@ def main(argv=None):
     sub = ap.add_subparsers(dest="what", required=True)
     p = sub.add_parser("prefill")
     p.add_argument("--small", action="store_true", help="3 launches of 2 x 2048 fp16 (profiling)")
-    sub.add_parser("gqa")
+    p = sub.add_parser("gqa")
+    p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     sub.add_parser("shared-prefix")
-    sub.add_parser("long-context")
+    p = sub.add_parser("long-context")
+    p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("kernel_bench needs a CUDA device")
     if args.what == "prefill":
         prefill(args.small)
     elif args.what == "gqa":
-        gqa()
+        gqa(args.partition_size)
     elif args.what == "shared-prefix":
         shared_prefix()
     else:
-        long_context()
+        long_context(args.partition_size)
 
 
 if __name__ == "__main__":
