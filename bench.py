@@ -12,7 +12,9 @@ and far larger than L2, so no flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One JSON line on rank 0.  Metric: KV bytes the attention reads per second
-(GB/s), with decode tokens/s and the HBM-roofline fraction beside it.
+(GB/s), with decode tokens/s and the HBM-roofline fraction beside it.  The
+step is timed as issued eagerly (the headline) and, beside it, replayed from
+a CUDA graph captured from the same calls.
 Multi-GPU runs are independent replicas (weak scaling): every rank owns its
 own 200 requests; the only collective is the max-over-ranks of the timing.
 `--impl reference` times the CPU oracle on a bounded sample of the same
@@ -162,10 +164,10 @@ def oracle_sample_case(seed, num_seqs_sample):
     return syn.decode_case(seed, lens, H, D, np.float16)
 
 
-def time_oracle(case, reps=1):
+def time_oracle(case, reps=1, threads=None):
     import oracle
 
-    cores = len(os.sched_getaffinity(0))
+    cores = threads or len(os.sched_getaffinity(0))
     os.environ["OMP_NUM_THREADS"] = str(cores)
     kp, vp = case["k_pool"].copy(), case["v_pool"].copy()
     slots = np.array([oracle.slot_of_c(case["block_tables"][s], int(L) - 1)
@@ -265,6 +267,13 @@ def run_ours(args):
 
     # every rank owns its own 200 requests (weak scaling): seed = rank
     lens, tables, nb = replica_workload(rank)
+    # the GPUs may be shared: refuse to start unless the pools fit
+    free, _ = torch.cuda.mem_get_info(dev)
+    need = 2 * args.layers * nb * H * BS * D * ELT + 4 * args.layers * S * H * D * ELT + (1 << 30)
+    if free < need:
+        print(json.dumps({"metric": METRIC, "error": f"not enough free HBM: {free / 2**30:.1f} GiB "
+                          f"free, {need / 2**30:.1f} GiB needed"}), flush=True)
+        raise SystemExit(3)
     pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
     n_layers = args.layers
     kpools, vpools = [], []
@@ -347,16 +356,22 @@ def run_ours(args):
     per_launch = algorithmic_bytes_per_launch(lens)
     achieved = per_launch / (decode_avg_ms * 1e-3) / 1e9
 
+    graph = run_graph(args, torch, step, stream, lens, n_layers, world, dev)
     e2e = None if args.no_e2e else run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens,
                                           ws, ps, world, dev)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         case = oracle_sample_case(0, 40)
         v, cores = time_oracle(case)
+        one = oracle_sample_case(0, 4)
+        v1, _ = time_oracle(one, threads=1)
         cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"one layer of the first 40 of the 200 requests "
                          f"({int(case['context_lens'].sum())} cached tokens), fp64 C oracle, "
-                         f"OpenMP over (sequence, head)"}
+                         f"OpenMP over (sequence, head)",
+               "single_thread": {"value": round(v1, 4), "unit": "GB/s", "cores": 1,
+                                 "sample": f"one layer of the first 4 requests "
+                                           f"({int(one['context_lens'].sum())} cached tokens)"}}
 
     if rank == 0:
         line = {
@@ -381,6 +396,7 @@ def run_ours(args):
                          "bytes_per_launch": per_launch,
                          "avg_launch_ms": round(decode_avg_ms, 5)},
             "gpu_launches": kernels_per_step * args.steps,
+            "graph": graph,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -389,6 +405,44 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_graph(args, torch, step, stream, lens, n_layers, world, dev):
+    """The same step (plan + one launch per layer) captured once into a CUDA
+    graph and replayed: host launch cost leaves the step.  None if capture is
+    refused (the eager number stands either way)."""
+    import torch.distributed as dist
+
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()  # warm the side stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            step()
+    except Exception as e:  # noqa: BLE001 - reported in the line, not hidden
+        torch.cuda.synchronize()
+        return {"error": f"capture failed: {type(e).__name__}: {e}"[:200]}
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    value = kv_bytes(lens) * n_layers * world / (ms * 1e-3) / 1e9
+    del g
+    return {"value": round(value, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
+            "decode_tokens_per_s": round(S * world / (ms * 1e-3), 1),
+            "launches_per_step": 1 + n_layers}
 
 
 def run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens, ws, ps, world, dev):

@@ -4,6 +4,7 @@
     python -m paged_kv_cache_478_b200.kernel_bench gqa
     python -m paged_kv_cache_478_b200.kernel_bench shared-prefix
     python -m paged_kv_cache_478_b200.kernel_bench long-context
+    python -m paged_kv_cache_478_b200.kernel_bench single-layer
 
 Each line printed is one JSON object.  These are the measurements behind the
 per-kernel tables of the design notes; the headline decode step is bench.py.
@@ -160,18 +161,20 @@ def shared_prefix():
                                                                   groups["max_shared_blocks"]),
                       dtype=torch.uint8, device="cuda")
     scale = 1 / math.sqrt(D)
-    t1 = _events_ms(lambda: pa.pa_decode_attention(pool, q, kp, vp, bt, cl, scale, out1, ws1), 50,
-                    flush=flush)
-    t2 = _events_ms(lambda: pa.pa_decode_attention_shared_prefix(pool, q, kp, vp, bt, cl, gd, scale,
-                                                                 out2, ws2), 50, flush=flush)
+    plain = lambda: pa.pa_decode_attention(pool, q, kp, vp, bt, cl, scale, out1, ws1)  # noqa: E731
+    shared = lambda: pa.pa_decode_attention_shared_prefix(  # noqa: E731
+        pool, q, kp, vp, bt, cl, gd, scale, out2, ws2)
+    rows = []
+    for l2, fl in (("flushed before every rep", flush), ("warm", None)):
+        rows.append(("plain decode", l2, _events_ms(plain, 50, flush=fl)))
+        rows.append(("shared-prefix path", l2, _events_ms(shared, 50, flush=fl)))
     _check()
     diff = (out1.float() - out2.float()).abs().max().item()
-    for name, ms in (("plain decode", t1), ("shared-prefix path", t2)):
+    for name, l2, ms in rows:
         print(json.dumps({"kernel": name, "sequences": S, "shared_prefix_tokens": P,
                           "us": round(ms * 1e3, 1), "logical_GBps": round(logical / ms / 1e6, 1),
                           "unique_GBps": round(unique / ms / 1e6, 1),
-                          "max_abs_diff_vs_plain": diff, "l2": "flushed before every rep"}),
-              flush=True)
+                          "max_abs_diff_vs_plain": diff, "l2": l2}), flush=True)
 
 
 def long_context(partition_size: int = 0):
@@ -198,6 +201,33 @@ def long_context(partition_size: int = 0):
                       "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
+def single_layer():
+    """One layer of 64 sequences, lengths uniform in [1, 2048], 32 heads x 128
+    fp16, the pool exactly the used blocks at random places; the new token is
+    appended and attended in one launch (about 1.1 GB of K/V, larger than L2)."""
+    S, H, D = 64, 32, 128
+    lens = syn.single_layer_lengths(0, S)
+    tables, nb = syn.full_step_tables(0, lens)
+    kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 1)
+    syn.fill_normal_device(vp, 2)
+    q = torch.randn((S, H, D), dtype=torch.float16, device="cuda")
+    kn, vn = torch.randn_like(q), torch.randn_like(q)
+    pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty_like(q)
+    ms = _events_ms(lambda: pa.pa_decode_append_attention(
+        pool, q, kn, vn, kp, vp, bt, cl, 1 / math.sqrt(D), out, ws), 50)
+    _check()
+    kv_bytes = int(lens.sum()) * H * D * 2 * 2
+    print(json.dumps({"kernel": "decode (single layer, plan + append + attend)", "sequences": S,
+                      "cached_tokens": int(lens.sum()), "us": round(ms * 1e3, 1),
+                      "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     sub = ap.add_subparsers(dest="what", required=True)
@@ -208,6 +238,7 @@ def main(argv=None):
     sub.add_parser("shared-prefix")
     p = sub.add_parser("long-context")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
+    sub.add_parser("single-layer")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("kernel_bench needs a CUDA device")
@@ -217,8 +248,10 @@ def main(argv=None):
         gqa(args.partition_size)
     elif args.what == "shared-prefix":
         shared_prefix()
-    else:
+    elif args.what == "long-context":
         long_context(args.partition_size)
+    else:
+        single_layer()
 
 
 if __name__ == "__main__":
