@@ -761,7 +761,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
   a.scale_log2 = scale * 1.4426950408889634f;
   const int64_t pairs = (max_new_tokens + 255) / 256;  // two 128-query tiles per CTA
   const int64_t hq = (int64_t)pool->heads * pool->q_per_kv;
-  if (pairs > INT32_MAX || hq > 65535 || num_seqs > 65535)
+  if (pairs > 65535 || hq > INT32_MAX || num_seqs > 65535)
     return fail(PA_ERR_INVALID_ARG, "prefill: grid too large");
   if ((int64_t)pool->num_blocks * pool->heads * kBlock > INT32_MAX)
     return fail(PA_ERR_INVALID_ARG, "prefill: pool rows exceed the tensor-copy coordinate range");
@@ -770,7 +770,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
   if ((st = encode_pool_map(*dev, &tk, k_pool, pool)) != PA_OK ||
       (st = encode_pool_map(*dev, &tv, v_pool, pool)) != PA_OK)
     return st;
-  const dim3 grid((unsigned)pairs, (unsigned)hq, (unsigned)num_seqs);
+  const dim3 grid((unsigned)hq, (unsigned)num_seqs, (unsigned)pairs);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = pool->dtype == PA_BF16;
   cudaError_t e;

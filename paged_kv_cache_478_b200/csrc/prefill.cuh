@@ -61,7 +61,7 @@ struct PrefillArgs {
   int32_t heads;     // KV heads
   int32_t q_per_kv;  // query heads per KV head
   int32_t max_context_len;
-  int32_t q_pairs;   // 256-query units per sequence in the grid (blockIdx.x range)
+  int32_t q_pairs;   // 256-query units per sequence in the grid (blockIdx.z range)
   float scale_log2;
 };
 
@@ -285,8 +285,10 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* smem = prefill_smem + ((1024u - (smem_addr(prefill_smem) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
 
-  // heaviest query pairs (latest positions, most keys) first
-  const int qt = a.q_pairs - 1 - (int)blockIdx.x, hq = blockIdx.y, s = blockIdx.z;
+  // grid (query head, sequence, query pair) with the pair slowest: CTAs start
+  // in linear order, so every sequence's and head's latest pairs (most keys)
+  // go first and the lightest fill the last wave
+  const int hq = blockIdx.x, s = blockIdx.y, qt = a.q_pairs - 1 - (int)blockIdx.z;
   const int q0 = a.query_start[s];
   const int n = a.query_start[s + 1] - q0;
   if (n <= 0 || qt * 2 * BM >= n) return;
