@@ -68,7 +68,7 @@ CASES = [(1, 1), (17, 17), (200, 64), (300, 300), (1000, 129), (128, 128), (2048
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [128, 64])
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
 def test_prefill_matches_the_oracle(dtype, head_dim, group):
     c = _case(70 + group, CASES, 2, group, head_dim, dtype)
     out = torch.empty_like(c["q"])
