@@ -5,6 +5,7 @@
     python -m paged_kv_cache_478_b200.kernel_bench shared-prefix
     python -m paged_kv_cache_478_b200.kernel_bench long-context
     python -m paged_kv_cache_478_b200.kernel_bench single-layer
+    python -m paged_kv_cache_478_b200.kernel_bench cache-ops
 
 Each line printed is one JSON object.  These are the measurements behind the
 per-kernel tables of the design notes; the headline decode step is bench.py.
@@ -43,6 +44,25 @@ def _events_ms(fn, reps: int, warmup: int = 3, flush: torch.Tensor | None = None
         pairs.append((e0, e1))
     torch.cuda.synchronize()
     return float(np.median([e0.elapsed_time(e1) for e0, e1 in pairs]))
+
+
+def _graph_us(fn, launches: int = 50, reps: int = 20) -> float:
+    """Device microseconds per call of a short kernel: `launches` calls are
+    captured into one CUDA graph and replayed, so host launch cost (larger
+    than these kernels) stays out; median over reps."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(launches):
+            fn()
+    ms = _events_ms(g.replay, reps)
+    del g
+    return ms * 1e3 / launches
 
 
 def _check():
@@ -228,6 +248,39 @@ def single_layer():
                       "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
+def cache_ops():
+    """reshape_and_cache and copy_blocks at the sizes of the workloads: one
+    decode step's new tokens (200), a long fill (32 768 tokens), and the
+    copy-on-write of config 3 (127 block pairs); 32 heads x 128 fp16."""
+    H, D = 32, 128
+    nb = 4096
+    kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
+    vp = torch.empty_like(kp)
+    syn.fill_normal_device(kp, 1)
+    syn.fill_normal_device(vp, 2)
+    pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
+    rng = np.random.default_rng(0)
+    for T in (200, 32768):
+        slots = torch.from_numpy(rng.permutation(nb * 16)[:T].astype(np.int32)).cuda()
+        kn = torch.randn((T, H, D), dtype=torch.float16, device="cuda")
+        vn = torch.randn_like(kn)
+        us = _graph_us(lambda: pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp),
+                       launches=50 if T <= 1024 else 5)
+        _check()
+        moved = 2 * 2 * T * H * D * 2  # K and V, read + written
+        print(json.dumps({"kernel": "reshape_and_cache", "tokens": T, "us": round(us, 2),
+                          "bytes_moved": moved, "GBps": round(moved / us / 1e3, 1)}), flush=True)
+    perm = rng.permutation(nb)[:254].astype(np.int32)
+    pairs = torch.from_numpy(perm.reshape(127, 2)).cuda()
+    us = _graph_us(lambda: pa.pa_copy_blocks(pool, kp, vp, pairs))
+    _check()
+    moved = 2 * 2 * 127 * H * 16 * D * 2  # K and V blocks, read + written
+    print(json.dumps({"kernel": "copy_blocks", "pairs": 127, "us": round(us, 2), "bytes_moved": moved,
+                      "GBps": round(moved / us / 1e3, 1),
+                      "l2": "warm: the 32.5 MB of source blocks stay in L2 across replays"}),
+          flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     sub = ap.add_subparsers(dest="what", required=True)
@@ -239,6 +292,7 @@ def main(argv=None):
     p = sub.add_parser("long-context")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     sub.add_parser("single-layer")
+    sub.add_parser("cache-ops")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("kernel_bench needs a CUDA device")
@@ -250,8 +304,10 @@ def main(argv=None):
         shared_prefix()
     elif args.what == "long-context":
         long_context(args.partition_size)
-    else:
+    elif args.what == "single-layer":
         single_layer()
+    else:
+        cache_ops()
 
 
 if __name__ == "__main__":
