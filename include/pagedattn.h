@@ -254,8 +254,9 @@ pa_status pa_decode_attention_shared_prefix(
  * must already be in the pool (pa_reshape_and_cache).  Query i sees tokens
  * 0..its position.  max_new_tokens bounds every n_s (launch sizing).
  * Runs on tcgen05 tensor cores with TMEM accumulators; fp16/bf16 pools,
- * head_dim 64 or 128.  A context length below n_s or above the table raises
- * PA_DEVERR_CONTEXT_LEN and that sequence is skipped.
+ * head_dim 64 or 128.  A context length below n_s or above the table, or
+ * n_s above max_new_tokens, raises PA_DEVERR_CONTEXT_LEN and that sequence is
+ * skipped (its rows of out are not written).
  */
 pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,
                                const void* v_pool, const int32_t* block_tables,

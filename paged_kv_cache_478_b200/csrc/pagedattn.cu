@@ -766,6 +766,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
   if ((int64_t)pool->num_blocks * pool->heads * kBlock > INT32_MAX)
     return fail(PA_ERR_INVALID_ARG, "prefill: pool rows exceed the tensor-copy coordinate range");
   a.q_pairs = (int32_t)pairs;
+  a.max_new_tokens = max_new_tokens;
   CUtensorMap tk, tv;
   if ((st = encode_pool_map(*dev, &tk, k_pool, pool)) != PA_OK ||
       (st = encode_pool_map(*dev, &tv, v_pool, pool)) != PA_OK)

@@ -130,3 +130,15 @@ def test_prefill_ignores_poisoned_rows_past_the_context(dtype):
     assert pa.pa_device_errors() == 0
     assert torch.isfinite(out.float()).all()
     assert_parity(out, c["ref"], f"prefill {dtype} with NaN past the context")
+
+
+def test_prefill_skips_and_reports_a_sequence_beyond_max_new_tokens():
+    """max_new_tokens sizes the launch; a sequence with more new tokens than
+    that is reported and left untouched, the others still run."""
+    c = _case(83, [(300, 300), (40, 20)], 2, 1, 128, "f16")
+    out = torch.zeros_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], c["qs"],
+                            c["scale"], out, 256)  # sequence 0 has 300 > 256
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
+    assert torch.count_nonzero(out[:300]) == 0
+    assert_parity(out[300:], c["ref"][300:], "the sequence within the bound still runs")
