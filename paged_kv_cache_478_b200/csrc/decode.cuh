@@ -1,4 +1,5 @@
-// Paged decode attention for sm_100a: work plan, partition kernel, split-K merge.
+// Paged decode attention for sm_100a: partition kernel and split-K merge (the
+// arguments and the work plan are in plan.cuh).
 //
 // The method: "PagedAttention" (e-fortepiano.pl wiki mirror), "Formulació
 // matemàtica" -- the attention of one query token, computed block by block
@@ -43,159 +44,9 @@
 
 #include "device_utils.cuh"
 #include "pagedattn.h"
+#include "plan.cuh"
 
 namespace pa {
-
-constexpr int kBlock = 16;  // tokens per physical block
-
-struct PlanHeader {
-  int32_t num_pairs;     // (sequence, partition) pairs
-  int32_t num_items;     // num_pairs * head_groups
-  int32_t work_counter;  // next item index to hand out
-  int32_t done_counter;  // CTAs that have left the work loop
-};
-
-struct DecodeArgs {
-  const void* q;
-  const void* k_pool;
-  const void* v_pool;
-  const int32_t* block_tables;
-  const int32_t* context_lens;
-  void* out;
-  PlanHeader* plan;
-  int32_t* lens;    // [S] clamped context lengths
-  int32_t* nparts;  // [S] partial results per sequence (>= 1): own partitions + shared chunks
-  int32_t* nitems;  // [S] own partitions (work items whose arrival triggers the merge)
-  int32_t* base;    // [S] first token of the sequence's own part (after its shared prefix)
-  int32_t* shared_of;  // [S] shared-prefix group of the sequence, or -1
-  // shared-prefix groups (null when there are none): CSR members, shared leading blocks
-  const int32_t* group_offsets;
-  const int32_t* group_members;
-  const int32_t* group_blocks;
-  int32_t num_groups;
-  int32_t max_shared_blocks;
-  int32_t shared_chunk;  // shared blocks per partial result
-  int2* pairs;      // [S * max_parts] work pairs (s, p)
-  float2* part_ml;  // [S][H][max_parts] (running max in log2 units, sum of weights)
-  float* part_acc;  // [S][H][max_parts][D] unnormalised partial outputs
-  int32_t* merge_cnt;  // [S][head_groups] partitions finished (re-armed to 0 by the merger)
-  const void* k_new;   // [S][H][D] token appended at position L-1, or null (no append)
-  const void* v_new;
-  uint32_t* err;
-  int64_t num_blocks;
-  int32_t max_blocks_per_seq;
-  int32_t num_seqs;
-  int32_t heads;        // KV heads in the pool
-  int32_t q_per_kv;     // query heads per KV head (1 = MHA; GQA/MQA otherwise)
-  int32_t head_groups;  // work items per (sequence, partition)
-  int32_t partition_size;
-  int32_t max_parts;
-  int32_t max_context_len;
-  float scale_log2;  // scale * log2(e)
-};
-
-// ---- plan: one CTA orders the work ------------------------------------------------
-
-__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
-  extern __shared__ int32_t bucket[];  // [nb + 1]: index 0 = sequences with no own tokens
-  __shared__ int32_t n_full;
-  const int PS = a.partition_size;
-  const int nb = PS / kBlock;
-  for (int i = threadIdx.x; i <= nb; i += blockDim.x) bucket[i] = 0;
-  if (threadIdx.x == 0) n_full = 0;
-  const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
-  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
-    int L = a.context_lens[s];
-    if (L < 0 || L > cap) {
-      atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-      L = L < 0 ? 0 : cap;
-    }
-    a.lens[s] = L;
-    a.shared_of[s] = -1;
-    for (int g = 0; g < a.head_groups; ++g) a.merge_cnt[(int64_t)s * a.head_groups + g] = 0;
-  }
-  __syncthreads();
-  // shared-prefix groups: a member joins if its table starts with the first
-  // member's blocks and it is long enough; anything else is reported and the
-  // sequence attends to its whole context on its own
-  if (a.group_offsets != nullptr) {
-    // groups in turn, their members spread over the CTA's threads
-    for (int g = 0; g < a.num_groups; ++g) {
-      const int m0 = a.group_offsets[g], m1 = a.group_offsets[g + 1];
-      const int nbk = a.group_blocks[g];
-      if (m1 <= m0 || nbk <= 0) continue;
-      if (nbk > a.max_shared_blocks || nbk > a.max_blocks_per_seq || m0 < 0) {
-        if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-        continue;
-      }
-      const int rep = a.group_members[m0];
-      if (rep < 0 || rep >= a.num_seqs || a.lens[rep] < nbk * kBlock) {
-        if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-        continue;
-      }
-      const int32_t* rt = a.block_tables + (int64_t)rep * a.max_blocks_per_seq;
-      // one warp per member: its lanes compare 32 table entries at a time
-      const int lane = threadIdx.x & 31;
-      for (int m = m0 + (threadIdx.x >> 5); m < m1; m += blockDim.x >> 5) {
-        const int s = a.group_members[m];
-        bool ok = s >= 0 && s < a.num_seqs && a.lens[s] >= nbk * kBlock;
-        if (ok) {
-          const int32_t* t = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-          int diff = 0;
-          for (int j = lane; j < nbk; j += 32) diff |= t[j] ^ rt[j];
-          ok = !__any_sync(kFullMask, diff != 0);
-        }
-        if (lane == 0) {
-          if (!ok) {
-            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-          } else if (atomicCAS(&a.shared_of[s], -1, g) != -1) {
-            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
-          }
-        }
-      }
-    }
-  }
-  __syncthreads();
-  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
-    const int L = a.lens[s];
-    const int g = a.shared_of[s];
-    const int sb = g >= 0 ? a.group_blocks[g] : 0;
-    const int base = sb * kBlock;
-    const int U = L - base;  // the sequence's own tokens
-    const int full = U / PS, rem = U % PS;
-    const int ni = max(1, full + (rem > 0 ? 1 : 0));
-    a.base[s] = base;
-    a.nitems[s] = ni;
-    a.nparts[s] = ni + (sb > 0 ? (sb + a.shared_chunk - 1) / a.shared_chunk : 0);
-    if (full > 0) {
-      const int pos = atomicAdd(&n_full, full);
-      for (int p = 0; p < full; ++p) a.pairs[pos + p] = make_int2(s, p);
-    }
-    if (U == 0 || rem > 0) atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = n_full;
-    for (int b = nb; b >= 0; --b) {  // biggest remainders first, empty ones last
-      const int c = bucket[b];
-      bucket[b] = run;
-      run += c;
-    }
-    a.plan->num_pairs = run;
-    a.plan->num_items = run * a.head_groups;
-    a.plan->work_counter = 0;
-    a.plan->done_counter = 0;
-  }
-  __syncthreads();
-  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
-    const int U = a.lens[s] - a.base[s];
-    const int rem = U % PS;
-    if (U == 0 || rem > 0) {
-      const int pos = atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
-      a.pairs[pos] = make_int2(s, U / PS);
-    }
-  }
-}
 
 // ---- transpose-reduce of NCH partial dot products over LPR lanes --------------------
 // Step with xor-mask M halves the values a lane carries: the lane keeps one

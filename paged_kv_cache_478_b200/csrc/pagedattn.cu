@@ -689,6 +689,7 @@ pa_status pa_decode_attention_shared_prefix(
     a.group_members = group_members;
     a.group_blocks = group_blocks;
     a.num_groups = num_groups;
+    a.max_group_size = max_group_size;
   }
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -308,3 +308,40 @@ def test_shared_prefix_groups_with_gqa_and_a_bad_member(dtype, group):
                                          _groups_to_device(groups), 1 / math.sqrt(D), out, ws)
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN  # the planted member
     assert_parity(out, ref, f"shared prefix {dtype} G={group}")
+
+
+def test_shared_prefix_group_larger_than_max_group_size():
+    """A group with more members than max_group_size (the launch covers that
+    many) is reported, and its members still get the right answer alone."""
+    rng = np.random.default_rng(61)
+    H, D = 2, 128
+    lens = np.array([400, 333, 321, 700, 1024, 250], dtype=np.int32)
+    nb = 300
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((6, 64), -1, dtype=np.int32)
+    shared = perm[:20]
+    pos = 20
+    for s, L in enumerate(lens):
+        n = math.ceil(int(L) / 16)
+        pre = shared if s < 5 else np.zeros(0, np.int32)
+        tables[s, :len(pre)] = pre
+        tables[s, len(pre):n] = perm[pos:pos + n - len(pre)]
+        pos += n - len(pre)
+    groups = pa.pa_find_shared_prefixes(tables, lens)
+    assert groups["num_groups"] == 1 and groups["offsets"].tolist() == [0, 5]
+    groups["max_group_size"] = 3  # the group has 5 members
+    shape = (nb, H, BS, D)
+    kt = torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
+    vt = torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
+    qt = torch.from_numpy(rng.standard_normal((6, H, D)).astype(np.float16))
+    ref = oracle.decode_attention(qt.numpy(), kt.numpy(), vt.numpy(), tables, lens,
+                                  1 / math.sqrt(D))
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    q = qt.cuda()
+    out = torch.empty_like(q)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(pool, 6, 64, 20),
+                     dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention_shared_prefix(pool, q, kt.cuda(), vt.cuda(), dev(tables), dev(lens),
+                                         _groups_to_device(groups), 1 / math.sqrt(D), out, ws)
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
+    assert_parity(out, ref, "oversized group attends alone")
