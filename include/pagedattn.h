@@ -225,9 +225,10 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
  * log-sum-exp.  fp16/bf16 pools only (PA_ERR_UNSUPPORTED for fp32).
  * max_group_size and max_shared_blocks bound the group sizes and
  * group_blocks (launch sizing); a group beyond either bound is reported
- * (PA_DEVERR_CONTEXT_LEN) and its members attend alone.  A member that is too short, holds
- * different blocks or belongs to two groups raises PA_DEVERR_CONTEXT_LEN and
- * attends to its whole context on its own, so the result stays correct.
+ * (PA_DEVERR_CONTEXT_LEN) and its members attend alone.  A member that is
+ * too short, holds different blocks or belongs to two groups raises
+ * PA_DEVERR_CONTEXT_LEN and attends to its whole context on its own, so the
+ * result stays correct.
  * Workspace: pa_decode_shared_prefix_workspace_bytes (max_shared_blocks
  * extra slots per head).  pa_find_shared_prefixes builds groups from host
  * block tables.
