@@ -6,6 +6,7 @@
     python -m paged_kv_cache_478_b200.kernel_bench long-context
     python -m paged_kv_cache_478_b200.kernel_bench single-layer
     python -m paged_kv_cache_478_b200.kernel_bench cache-ops
+    python -m paged_kv_cache_478_b200.kernel_bench decode-dtypes
 
 Each line printed is one JSON object.  These are the measurements behind the
 per-kernel tables of the design notes; the headline decode step is bench.py.
@@ -116,21 +117,26 @@ def prefill(small: bool):
                           "ms": round(ms, 4), "TFLOPs": round(flops / ms / 1e9, 1)}), flush=True)
 
 
-def gqa(partition_size: int = 0):
+_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def gqa(partition_size: int = 0, dtype: str = "f16"):
     S, HK, D = 200, 8, 128
+    dt = _DTYPES[dtype]
+    elt = torch.tensor([], dtype=dt).element_size()
     lens = syn.full_step_lengths(0, S)
     tables, nb = syn.full_step_tables(0, lens)
-    kp = torch.empty((nb, HK, 16, D), dtype=torch.float16, device="cuda")
+    kp = torch.empty((nb, HK, 16, D), dtype=dt, device="cuda")
     vp = torch.empty_like(kp)
     syn.fill_normal_device(kp, 1)
     syn.fill_normal_device(vp, 2)
     bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
-    kv_bytes = int(lens.sum()) * HK * D * 2 * 2
+    kv_bytes = int(lens.sum()) * HK * D * elt * 2
     for G in (1, 2, 4, 8):
-        pool = pa.pa_pool_create(nb, 16, HK, D, torch.float16)
+        pool = pa.pa_pool_create(nb, 16, HK, D, dt)
         pa.pa_pool_set_query_heads(pool, HK * G)
-        q = torch.randn((S, HK * G, D), dtype=torch.float16, device="cuda")
-        kn = torch.randn((S, HK, D), dtype=torch.float16, device="cuda")
+        q = torch.randn((S, HK * G, D), dtype=dt, device="cuda")
+        kn = torch.randn((S, HK, D), dtype=dt, device="cuda")
         vn = torch.randn_like(kn)
         out = torch.empty_like(q)
         ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, partition_size),
@@ -140,7 +146,7 @@ def gqa(partition_size: int = 0):
             pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size),
             50)
         _check()
-        print(json.dumps({"kernel": "decode (GQA)", "q_per_kv": G, "kv_heads": HK,
+        print(json.dumps({"kernel": "decode (GQA)", "dtype": dtype, "q_per_kv": G, "kv_heads": HK,
                           "partition_size": partition_size or "auto",
                           "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}),
               flush=True)
@@ -281,6 +287,36 @@ def cache_ops():
           flush=True)
 
 
+def decode_dtypes():
+    """One layer of the full decode step (200 requests, full-step lengths, 32
+    heads x 128) for each pool dtype: planned append + attend."""
+    S, H, D = 200, 32, 128
+    lens = syn.full_step_lengths(0, S)
+    tables, nb = syn.full_step_tables(0, lens)
+    bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    for name, dt in _DTYPES.items():
+        elt = torch.tensor([], dtype=dt).element_size()
+        kp = torch.empty((nb, H, 16, D), dtype=dt, device="cuda")
+        vp = torch.empty_like(kp)
+        syn.fill_normal_device(kp, 1)
+        syn.fill_normal_device(vp, 2)
+        q = torch.randn((S, H, D), dtype=dt, device="cuda")
+        kn, vn = torch.randn_like(q), torch.randn_like(q)
+        out = torch.empty_like(q)
+        pool = pa.pa_pool_create(nb, 16, H, D, dt)
+        ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
+                         device="cuda")
+        pa.pa_decode_plan(pool, cl, tables.shape[1], ws)
+        ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
+            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws), 30)
+        _check()
+        kv_bytes = int(lens.sum()) * H * D * elt * 2
+        print(json.dumps({"kernel": "decode (one full-step layer)", "dtype": name,
+                          "us": round(ms * 1e3, 1), "kv_bytes": kv_bytes,
+                          "kv_GBps": round(kv_bytes / ms / 1e6, 1)}), flush=True)
+        del kp, vp
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     sub = ap.add_subparsers(dest="what", required=True)
@@ -288,26 +324,30 @@ def main(argv=None):
     p.add_argument("--small", action="store_true", help="3 launches of 2 x 2048 fp16 (profiling)")
     p = sub.add_parser("gqa")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
+    p.add_argument("--dtype", choices=sorted(_DTYPES), default="f16")
     sub.add_parser("shared-prefix")
     p = sub.add_parser("long-context")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     sub.add_parser("single-layer")
     sub.add_parser("cache-ops")
+    sub.add_parser("decode-dtypes")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("kernel_bench needs a CUDA device")
     if args.what == "prefill":
         prefill(args.small)
     elif args.what == "gqa":
-        gqa(args.partition_size)
+        gqa(args.partition_size, args.dtype)
     elif args.what == "shared-prefix":
         shared_prefix()
     elif args.what == "long-context":
         long_context(args.partition_size)
     elif args.what == "single-layer":
         single_layer()
-    else:
+    elif args.what == "cache-ops":
         cache_ops()
+    else:
+        decode_dtypes()
 
 
 if __name__ == "__main__":
