@@ -580,42 +580,60 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < BN; ++c)
             if (!row_valid || j * BN + c > pos) sc[c] = masked_raw;
         }
-        // row max of the scaled scores (8 independent chains)
+        // bf16: the row's max and its weights against the current reference
+        // max are computed in one pass (the max on the ALU pipe while the
+        // exp2s run on the multi-function unit); only if the max passed the
+        // reference by more than 2^8 -- on a row's first tile, and rarely
+        // after -- does the reference move and the warp redo the row from S,
+        // still in TMEM.  That measured +19 % for bf16, whose high/residual
+        // split keeps the ALU busiest, and -1 % for fp16, which finds the max
+        // first.
+        const float2 sl2v = make_float2(sl2, sl2);
+        auto weights = [&](float mb) {
+          const float2 nmb = make_float2(-mb, -mb);
+#pragma unroll
+          for (int i = 0; i < BN / 2; ++i) {
+            const float2 x = __ffma2_rn(sv[i], sl2v, nmb);
+            sv[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          }
+        };
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = sc[i];
+        const bool ahead = kSplitP<T> && __all_sync(kFullMask, m_used != -INFINITY);
         if (sl2 >= 0.f) {
 #pragma unroll
           for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sc[c]);
-#pragma unroll
-          for (int i = 4; i >= 1; i >>= 1)
-#pragma unroll
-            for (int k = 0; k < i; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + i]);
         } else {
 #pragma unroll
           for (int c = 8; c < BN; ++c) mx8[c & 7] = fminf(mx8[c & 7], sc[c]);
-#pragma unroll
-          for (int i = 4; i >= 1; i >>= 1)
-#pragma unroll
-            for (int k = 0; k < i; ++k) mx8[k] = fminf(mx8[k], mx8[k + i]);
         }
-        const float mraw = mx8[0];
-        const float m_tile = sl2 == 0.f ? 0.f : mraw * sl2;
+        if (ahead) weights(m_used);  // independent of the max: overlaps it
+#pragma unroll
+        for (int i = 4; i >= 1; i >>= 1)
+#pragma unroll
+          for (int k = 0; k < i; ++k)
+            mx8[k] = sl2 >= 0.f ? fmaxf(mx8[k], mx8[k + i]) : fminf(mx8[k], mx8[k + i]);
+        const float m_tile = sl2 == 0.f ? 0.f : mx8[0] * sl2;
         // move the reference max only when a weight would exceed 2^8
         const bool move = m_tile > m_used + 8.f;
         float alpha = 1.f;
-        if (move) {
-          alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - m_tile);
-          m_used = m_tile;
-        }
-        const float mb = m_used == -INFINITY ? 0.f : m_used;
-        const float2 sl2v = make_float2(sl2, sl2), nmb = make_float2(-mb, -mb);
-        // weights in fp32: exp2 on the multi-function unit (4 per clock per
-        // sub-partition, in step with the tensor core's work on the tile)
+        if (__any_sync(kFullMask, move) || !ahead) {
+          if (move) {
+            alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - m_tile);
+            m_used = m_tile;
+          }
+          if (ahead) {  // the weights above are stale: S again from TMEM
 #pragma unroll
-        for (int i = 0; i < BN / 2; ++i) {
-          const float2 x = __ffma2_rn(sv[i], sl2v, nmb);
-          sv[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            for (int c0 = 0; c0 < BN; c0 += 32) tmem_ld32_nowait(s_addr + c0, sc + c0);
+            tmem_wait_ld();
+            if (need_mask) {
+#pragma unroll
+              for (int c = 0; c < BN; ++c)
+                if (!row_valid || j * BN + c > pos) sc[c] = masked_raw;
+            }
+          }
+          weights(m_used == -INFINITY ? 0.f : m_used);
         }
         if (need_mask) {  // a zero scale keeps masked scores finite: select them out
 #pragma unroll
