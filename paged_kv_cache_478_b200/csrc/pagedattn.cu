@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -49,6 +50,16 @@ struct DeviceState {
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
+
+// One NVTX range per C-ABI call that launches work, named after the call, so
+// a timeline profiler shows each call around its kernels.  Header-only NVTX:
+// without an attached tool the push and pop cost a few nanoseconds.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 pa_status cuda_fail(cudaError_t e, const char* what) {
   char buf[256];
@@ -396,6 +407,7 @@ pa_status pa_pool_set_query_heads(pa_pool* pool, int32_t num_q_heads) {
 pa_status pa_reshape_and_cache(const pa_pool* pool, const void* k_new, const void* v_new,
                                const int32_t* slot_mapping, int32_t num_tokens, void* k_pool,
                                void* v_pool, void* stream) {
+  CallRange range("pa_reshape_and_cache");
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: num_tokens < 0");
@@ -563,6 +575,7 @@ pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32
                          int32_t max_blocks_per_seq, int32_t max_context_len,
                          int32_t partition_size, void* workspace, size_t workspace_bytes,
                          void* stream) {
+  CallRange range("pa_decode_plan");
   if (num_seqs == 0) return check_pool(pool);
   if (!context_lens) return fail(PA_ERR_INVALID_ARG, "pa_decode_plan: context_lens is null");
   DecodeArgs a;
@@ -580,6 +593,7 @@ pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const 
                                       int32_t max_context_len, float scale, void* out,
                                       void* workspace, size_t workspace_bytes,
                                       int32_t partition_size, void* stream) {
+  CallRange range("pa_decode_attention_planned");
   if (num_seqs == 0) return check_pool(pool);
   pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
   if (st != PA_OK) return st;
@@ -598,6 +612,7 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
                               int32_t num_seqs, int32_t max_context_len, float scale, void* out,
                               void* workspace, size_t workspace_bytes, int32_t partition_size,
                               void* stream) {
+  CallRange range("pa_decode_attention");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention: num_seqs < 0");
   if (num_seqs == 0) return check_pool(pool);
   pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
@@ -622,6 +637,7 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
                                              int32_t max_context_len, float scale, void* out,
                                              void* workspace, size_t workspace_bytes,
                                              int32_t partition_size, void* stream) {
+  CallRange range("pa_decode_append_attention_planned");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode append: num_seqs < 0");
   if (num_seqs == 0) return check_pool(pool);
   pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
@@ -647,6 +663,7 @@ pa_status pa_decode_append_attention(const pa_pool* pool, const void* q, const v
                                      int32_t max_context_len, float scale, void* out,
                                      void* workspace, size_t workspace_bytes,
                                      int32_t partition_size, void* stream) {
+  CallRange range("pa_decode_append_attention");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode append: num_seqs < 0");
   if (num_seqs == 0) return check_pool(pool);
   pa_status st = pa_decode_plan(pool, context_lens, num_seqs, max_blocks_per_seq,
@@ -666,6 +683,7 @@ pa_status pa_decode_attention_shared_prefix(
     const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
     int32_t max_shared_blocks, int32_t max_context_len, float scale, void* out, void* workspace,
     size_t workspace_bytes, int32_t partition_size, void* stream) {
+  CallRange range("pa_decode_attention_shared_prefix");
   if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "shared prefix: negative size");
   if (num_seqs == 0) return check_pool(pool);
@@ -733,6 +751,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
                                const int32_t* query_start, int32_t num_seqs,
                                int32_t max_new_tokens, int32_t max_context_len, float scale,
                                void* out, void* stream) {
+  CallRange range("pa_prefill_attention");
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_seqs < 0 || max_new_tokens < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
@@ -787,6 +806,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
 
 pa_status pa_copy_blocks(const pa_pool* pool, void* k_pool, void* v_pool, const int32_t* pairs,
                          int32_t num_pairs, void* stream) {
+  CallRange range("pa_copy_blocks");
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
   if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: num_pairs < 0");
@@ -858,6 +878,7 @@ pa_status pa_decode_attention_static(const pa_pool* pool, const void* q, const v
                                      int32_t max_blocks_per_seq, const int32_t* context_lens,
                                      int32_t num_seqs, int32_t max_context_len, float scale,
                                      void* out, int32_t partition_size, void* stream) {
+  CallRange range("pa_decode_attention_static");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: num_seqs < 0");
   size_t need = 0;
   pa_status st = pa_decode_workspace_bytes(pool, num_seqs, max_blocks_per_seq, max_context_len,
