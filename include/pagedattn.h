@@ -256,14 +256,15 @@ pa_status pa_decode_attention_shared_prefix(
  * must already be in the pool (pa_reshape_and_cache).  Query i sees tokens
  * 0..its position.  max_new_tokens bounds every n_s (launch sizing).
  * Runs on tcgen05 tensor cores with TMEM accumulators; fp16/bf16 pools,
- * head_dim 64 or 128.  A context length below n_s or above the table, or
- * n_s above max_new_tokens, raises PA_DEVERR_CONTEXT_LEN and that sequence is
- * skipped (its rows of out are not written).
+ * head_dim 64 or 128.  num_tokens is the number of rows q and out hold.  A
+ * context length below n_s or above the table, n_s above max_new_tokens, or
+ * rows outside [0, num_tokens) raise PA_DEVERR_CONTEXT_LEN and that sequence
+ * is skipped (its rows of out are not written).
  */
 pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,
                                const void* v_pool, const int32_t* block_tables,
                                int32_t max_blocks_per_seq, const int32_t* context_lens,
-                               const int32_t* query_start, int32_t num_seqs,
+                               const int32_t* query_start, int32_t num_seqs, int32_t num_tokens,
                                int32_t max_new_tokens, int32_t max_context_len, float scale,
                                void* out, void* stream);
 

@@ -88,7 +88,7 @@ def lib():
                                                   sz, i32, vp],
             "pa_find_shared_prefixes": [vp, i32, vp, i32, i32, i32, vp, vp, vp, P(i32), P(i32),
                                         P(i32)],
-            "pa_prefill_attention": [P(pa_pool), vp, vp, vp, vp, i32, vp, vp, i32, i32, i32,
+            "pa_prefill_attention": [P(pa_pool), vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
                                      ctypes.c_float, vp, vp],
             "pa_copy_blocks": [P(pa_pool), vp, vp, vp, i32, vp],
             "pa_device_errors": [vp, P(ctypes.c_uint32)],
@@ -380,7 +380,7 @@ def pa_prefill_attention(pool, q, k_pool, v_pool, block_tables, context_lens, qu
         _check_pool_tensor(pool, v_pool, "v_pool"),
         _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev_ptr(context_lens, "context_lens", torch.int32),
-        _dev_ptr(query_start, "query_start", torch.int32), S, max_new_tokens, max_context_len,
+        _dev_ptr(query_start, "query_start", torch.int32), S, T, max_new_tokens, max_context_len,
         float(scale), _dev_ptr(out, "out", dt), _stream(stream)))
 
 

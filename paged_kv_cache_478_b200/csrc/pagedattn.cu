@@ -748,15 +748,16 @@ pa_status pa_decode_attention_shared_prefix(
 pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,
                                const void* v_pool, const int32_t* block_tables,
                                int32_t max_blocks_per_seq, const int32_t* context_lens,
-                               const int32_t* query_start, int32_t num_seqs,
+                               const int32_t* query_start, int32_t num_seqs, int32_t num_tokens,
                                int32_t max_new_tokens, int32_t max_context_len, float scale,
                                void* out, void* stream) {
   CallRange range("pa_prefill_attention");
   pa_status st = check_pool(pool);
   if (st != PA_OK) return st;
-  if (num_seqs < 0 || max_new_tokens < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+  if (num_seqs < 0 || num_tokens < 0 || max_new_tokens < 0 || max_blocks_per_seq <= 0 ||
+      max_context_len < 0)
     return fail(PA_ERR_INVALID_ARG, "prefill: bad size");
-  if (num_seqs == 0 || max_new_tokens == 0) return PA_OK;
+  if (num_seqs == 0 || max_new_tokens == 0 || num_tokens == 0) return PA_OK;
   if (pool->dtype == PA_F32)
     return fail(PA_ERR_UNSUPPORTED, "prefill: fp16 or bf16 pools only (tcgen05 kind::f16)");
   st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
@@ -787,6 +788,7 @@ pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k
     return fail(PA_ERR_INVALID_ARG, "prefill: pool rows exceed the tensor-copy coordinate range");
   a.q_pairs = (int32_t)pairs;
   a.max_new_tokens = max_new_tokens;
+  a.num_tokens = num_tokens;
   CUtensorMap tk, tv;
   if ((st = encode_pool_map(*dev, &tk, k_pool, pool)) != PA_OK ||
       (st = encode_pool_map(*dev, &tv, v_pool, pool)) != PA_OK)

@@ -63,6 +63,7 @@ struct PrefillArgs {
   int32_t max_context_len;
   int32_t q_pairs;   // 256-query units per sequence in the grid (blockIdx.z range)
   int32_t max_new_tokens;  // bound on every sequence's new tokens (the grid covers it)
+  int32_t num_tokens;      // rows of q and out
   float scale_log2;
 };
 
@@ -304,7 +305,8 @@ __global__ void __launch_bounds__(384, 1)
   const int hq = blockIdx.x, s = blockIdx.y, qt = a.q_pairs - 1 - (int)blockIdx.z;
   const int q0 = a.query_start[s];
   const int n = a.query_start[s + 1] - q0;
-  if (n > a.max_new_tokens) {  // beyond the launch's bound: skipped whole, reported once
+  // rows outside q / out, or beyond the launch's bound: skipped whole, reported once
+  if (n > a.max_new_tokens || (n > 0 && (q0 < 0 || q0 > a.num_tokens - n))) {
     if (qt == 0 && hq == 0 && threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
     return;
   }

@@ -142,3 +142,17 @@ def test_prefill_skips_and_reports_a_sequence_beyond_max_new_tokens():
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
     assert torch.count_nonzero(out[:300]) == 0
     assert_parity(out[300:], c["ref"][300:], "the sequence within the bound still runs")
+
+
+def test_prefill_skips_a_sequence_whose_rows_fall_outside_q():
+    """query_start is device data: a sequence whose rows run past the q/out
+    rows (num_tokens) is reported and skipped, and nothing outside is read or
+    written."""
+    c = _case(84, [(64, 32), (40, 20)], 2, 1, 128, "f16")
+    bad_qs = torch.tensor([0, 32, 60], dtype=torch.int32, device="cuda")  # 60 > 52 rows
+    out = torch.zeros_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], bad_qs,
+                            c["scale"], out, 32)
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
+    assert torch.count_nonzero(out[32:]) == 0
+    assert_parity(out[:32], c["ref"][:32], "the sequence inside q still runs")
