@@ -216,7 +216,8 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
  * pa_decode_attention, computed so that each shared block is read once for
  * all the sequences holding it.
  * Groups (device int32 arrays, CSR): members of group g are
- * group_members[group_offsets[g] .. group_offsets[g+1]); they all hold the
+ * group_members[group_offsets[g] .. group_offsets[g+1]) (num_members entries
+ * in all; offsets outside them reject the group); they all hold the
  * same physical blocks as the group's first member in their first
  * group_blocks[g] table entries, and those blocks are full (16 tokens).
  * A tensor-core kernel attends every member's query heads to the shared
@@ -242,7 +243,7 @@ pa_status pa_decode_attention_shared_prefix(
     const pa_pool* pool, const void* q, const void* k_pool, const void* v_pool,
     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
     int32_t num_seqs, const int32_t* group_offsets, const int32_t* group_members,
-    const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
+    int32_t num_members, const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
     int32_t max_shared_blocks, int32_t max_context_len, float scale, void* out, void* workspace,
     size_t workspace_bytes, int32_t partition_size, void* stream);
 

@@ -84,8 +84,8 @@ def lib():
                                            ctypes.c_float, vp, i32, vp],
             "pa_decode_shared_prefix_workspace_bytes": [P(pa_pool), i32, i32, i32, i32, i32, P(sz)],
             "pa_decode_attention_shared_prefix": [P(pa_pool), vp, vp, vp, vp, i32, vp, i32, vp, vp,
-                                                  vp, i32, i32, i32, i32, ctypes.c_float, vp, vp,
-                                                  sz, i32, vp],
+                                                  i32, vp, i32, i32, i32, i32, ctypes.c_float, vp,
+                                                  vp, sz, i32, vp],
             "pa_find_shared_prefixes": [vp, i32, vp, i32, i32, i32, vp, vp, vp, P(i32), P(i32),
                                         P(i32)],
             "pa_prefill_attention": [P(pa_pool), vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
@@ -353,11 +353,14 @@ def pa_decode_attention_shared_prefix(pool, q, k_pool, v_pool, block_tables, con
     ng = groups["num_groups"]
     gp = [_dev_ptr(groups[k], k, torch.int32) if ng > 0 else None
           for k in ("offsets", "members", "blocks")]
+    nm = groups["members"].numel() if ng > 0 else 0
+    if ng > 0 and (groups["offsets"].numel() != ng + 1 or groups["blocks"].numel() != ng):
+        raise ValueError("groups: offsets must have num_groups + 1 entries, blocks num_groups")
     _check(lib().pa_decode_attention_shared_prefix(
         ctypes.byref(pool), _dev_ptr(q, "q", dt), _check_pool_tensor(pool, k_pool, "k_pool"),
         _check_pool_tensor(pool, v_pool, "v_pool"),
         _dev_ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1],
-        _dev_ptr(context_lens, "context_lens", torch.int32), S, gp[0], gp[1], gp[2], ng,
+        _dev_ptr(context_lens, "context_lens", torch.int32), S, gp[0], gp[1], nm, gp[2], ng,
         groups["max_group_size"], groups["max_shared_blocks"], max_context_len, float(scale),
         _dev_ptr(out, "out", dt), _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), partition_size, _stream(stream)))

@@ -680,11 +680,12 @@ pa_status pa_decode_attention_shared_prefix(
     const pa_pool* pool, const void* q, const void* k_pool, const void* v_pool,
     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
     int32_t num_seqs, const int32_t* group_offsets, const int32_t* group_members,
-    const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
+    int32_t num_members, const int32_t* group_blocks, int32_t num_groups, int32_t max_group_size,
     int32_t max_shared_blocks, int32_t max_context_len, float scale, void* out, void* workspace,
     size_t workspace_bytes, int32_t partition_size, void* stream) {
   CallRange range("pa_decode_attention_shared_prefix");
-  if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0)
+  if (num_seqs < 0 || num_groups < 0 || num_members < 0 || max_group_size < 0 ||
+      max_shared_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "shared prefix: negative size");
   if (num_seqs == 0) return check_pool(pool);
   pa_status st = check_pool(pool);
@@ -707,6 +708,7 @@ pa_status pa_decode_attention_shared_prefix(
     a.group_members = group_members;
     a.group_blocks = group_blocks;
     a.num_groups = num_groups;
+    a.num_members = num_members;
     a.max_group_size = max_group_size;
   }
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
@@ -716,6 +718,7 @@ pa_status pa_decode_attention_shared_prefix(
     SharedPrefixArgs sp;
     sp.group_offsets = group_offsets;
     sp.group_members = group_members;
+    sp.num_members = num_members;
     sp.group_blocks = group_blocks;
     sp.num_groups = num_groups;
     const int rows = max_group_size * pool->q_per_kv;

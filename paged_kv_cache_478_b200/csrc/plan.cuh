@@ -41,6 +41,7 @@ struct DecodeArgs {
   // shared-prefix groups (null when there are none): CSR members, shared leading blocks
   const int32_t* group_offsets;
   const int32_t* group_members;
+  int32_t num_members;     // entries of group_members
   const int32_t* group_blocks;
   int32_t num_groups;
   int32_t max_shared_blocks;
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
       if (m1 <= m0 || nbk <= 0) continue;
       // a group beyond the launch's bounds would be covered only in part
       if (nbk > a.max_shared_blocks || nbk > a.max_blocks_per_seq || m0 < 0 ||
-          m1 - m0 > a.max_group_size) {
+          m1 > a.num_members || m1 - m0 > a.max_group_size) {
         if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
         continue;
       }

@@ -32,6 +32,7 @@ namespace pa {
 struct SharedPrefixArgs {
   const int32_t* group_offsets;  // [G+1] CSR offsets into group_members
   const int32_t* group_members;  // sequence ids
+  int32_t num_members;           // entries of group_members
   const int32_t* group_blocks;   // [G] shared leading blocks of each group
   int32_t num_groups;
   int32_t row_tiles;   // 64-row tiles per group (from the largest group)
@@ -69,7 +70,9 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
   const int rows_in_group = (m1 - m0) * G;
   if (m1 <= m0 || blk_lo >= blk_hi || row_tile * Cfg::ROWS >= rows_in_group) return;
   // groups the plan could not have accepted are skipped (their members attend alone)
-  if (m0 < 0 || nblocks > a.max_shared_blocks || nblocks > a.max_blocks_per_seq) return;
+  if (m0 < 0 || m1 > sp.num_members || m1 - m0 > a.max_group_size ||
+      nblocks > a.max_shared_blocks || nblocks > a.max_blocks_per_seq)
+    return;
   const int rep = sp.group_members[m0];  // any member's table names the shared blocks
   if (rep < 0 || rep >= a.num_seqs) return;
   const int HK = a.heads, HQ = a.heads * G;

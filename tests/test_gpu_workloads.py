@@ -345,3 +345,38 @@ def test_shared_prefix_group_larger_than_max_group_size():
                                          _groups_to_device(groups), 1 / math.sqrt(D), out, ws)
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
     assert_parity(out, ref, "oversized group attends alone")
+
+
+def test_shared_prefix_offsets_past_the_members_array():
+    """group_offsets is device data: offsets beyond the members array reject
+    the group (reported) without reading past the array."""
+    rng = np.random.default_rng(62)
+    H, D = 2, 128
+    lens = np.array([400, 333, 321, 700, 1024], dtype=np.int32)
+    nb = 300
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((5, 64), -1, dtype=np.int32)
+    pos = 20
+    for s, L in enumerate(lens):
+        n = math.ceil(int(L) / 16)
+        tables[s, :20] = perm[:20]
+        tables[s, 20:n] = perm[pos:pos + n - 20]
+        pos += n - 20
+    groups = pa.pa_find_shared_prefixes(tables, lens)
+    assert groups["offsets"].tolist() == [0, 5]
+    groups["members"] = groups["members"][:3]  # offsets say 5 members, the array holds 3
+    shape = (nb, H, BS, D)
+    kt = torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
+    vt = torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
+    qt = torch.from_numpy(rng.standard_normal((5, H, D)).astype(np.float16))
+    ref = oracle.decode_attention(qt.numpy(), kt.numpy(), vt.numpy(), tables, lens,
+                                  1 / math.sqrt(D))
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    q = qt.cuda()
+    out = torch.empty_like(q)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(pool, 5, 64, 20),
+                     dtype=torch.uint8, device="cuda")
+    pa.pa_decode_attention_shared_prefix(pool, q, kt.cuda(), vt.cuda(), dev(tables), dev(lens),
+                                         _groups_to_device(groups), 1 / math.sqrt(D), out, ws)
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
+    assert_parity(out, ref, "a rejected group's members attend alone")
