@@ -6,27 +6,30 @@
 // applies to every query; with 128 queries a tile the two products are dense
 // contractions, S = Q.K^T and O = P.V.
 //
-// One CTA = (sequence, query head, 256 new queries as two 128-row tiles) with
-// specialised warps:
+// A work item = (sequence, query head, 256 new queries as two 128-row tiles).
+// One persistent CTA per SM walks the items heaviest first, with specialised
+// warps:
 //   * warps 0-3 and 4-7: two softmax warpgroups, one per query tile; thread r
 //     of a group owns query row r (TMEM lane r).  Each reads its row of S
 //     (128 keys) from TMEM, applies the causal mask and the online softmax in
 //     fp32 (log2 domain) and writes its row of P (fp16/bf16 pairs) back over
-//     S in TMEM, where the P.V product takes its A operand from;
-//   * warp 8: the loader.  It streams the paged K and V rows of each 64-key
-//     tile with TMA tensor copies (one 16-row box per physical block and
-//     64-wide slice of head_dim, hardware 128-byte swizzle) into a ring of
-//     K/V stages; the valid V rows of a partly filled last block are copied
-//     by its lanes and the V rows past the context are zeroed;
+//     S in TMEM, where the P.V product takes its A operand from; at the end
+//     of an item it writes its rows of O out and frees O for the next item;
+//   * warp 8: the loader.  It loads each item's Q tiles and streams the paged
+//     K and V rows of each 128-key tile with TMA tensor copies (one 16-row box
+//     per physical block and 64-wide slice of head_dim, hardware 128-byte
+//     swizzle) into rings of K and V stages that run on across items; the
+//     valid V rows of a partly filled last block are copied by its lanes and
+//     the V rows past the context are zeroed;
 //   * warp 9: one thread issues the tensor-core products into TMEM and commits
 //     them to mbarriers.
 // The two query tiles share every K/V stage and take turns on the tensor core:
 // while one group runs its softmax, the MMA unit computes the other group's
 // P.V and next S.  Keeping P in TMEM leaves shared memory to the Q, K and V
 // operands, whose bandwidth bounds the products (128-key tiles halve the Q
-// re-reads per flop against 64-key ones).  The running max is only moved (and the row of O in TMEM
-// rescaled) when a score exceeds it by more than 2^8, which keeps every
-// weight at most 256 and makes the rescale rare.
+// re-reads per flop against 64-key ones).  The running max is only moved
+// (and the row of O in TMEM rescaled) when a score exceeds it by more than
+// 2^8, which keeps every weight at most 256 and makes the rescale rare.
 // Shared-memory operands are described by SW128 matrix descriptors (K-major
 // for Q and K; MN-major for V).  Every wait is bounded; a wait that gives
 // up stops the CTA's other roles, lets every copy and product already issued
@@ -61,7 +64,7 @@ struct PrefillArgs {
   int32_t heads;     // KV heads
   int32_t q_per_kv;  // query heads per KV head
   int32_t max_context_len;
-  int32_t q_pairs;   // 256-query units per sequence in the grid (blockIdx.z range)
+  int32_t q_pairs;   // 256-query units per sequence (work items per (sequence, head))
   int32_t max_new_tokens;  // bound on every sequence's new tokens (the grid covers it)
   int32_t num_tokens;      // rows of q and out
   float scale_log2;
@@ -80,10 +83,10 @@ struct PrefillConfig {
   static constexpr int LOAD_WARP = 8, MMA_WARP = 9;  // warps 10-11 only fill the warpgroup
   static constexpr int THREADS = 384;
   // Launched at 168 registers a thread (384 x 168 fit the register file);
-  // the loader/MMA warpgroup then drops to 72 and the softmax groups rise to
-  // 216: 256 x 216 + 128 x 72 = 64512 = 384 x 168 launched (per SM
+  // the loader/MMA warpgroup then drops to 104 and the softmax groups rise to
+  // 200: 256 x 200 + 128 x 104 = 64512 = 384 x 168 launched (per SM
   // sub-partition: two softmax warps and one other, 16128 of 16384).
-  static constexpr int REGS_LAUNCH = 168, REGS_SOFTMAX = 216, REGS_OTHER = 72;
+  static constexpr int REGS_LAUNCH = 168, REGS_SOFTMAX = 200, REGS_OTHER = 104;
   static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * REGS_LAUNCH, "register split");
   static constexpr int Q_BYTES = KB * BM * 128;
   static constexpr int KV_BYTES = KB * BN * 128;   // one stage of K or of V
@@ -91,11 +94,12 @@ struct PrefillConfig {
   static constexpr int OFF_K = OFF_Q + QT * Q_BYTES;            // [stage]
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;           // [stage]
   static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-  // mbarriers: q_full[2], K full/empty[NS], V full/empty[NS], s_full[2],
-  // p_full[2], o_done[2], fin
-  static constexpr int BAR_Q = 0, BAR_KF = 2, BAR_KE = BAR_KF + NS, BAR_VF = BAR_KE + NS,
-                       BAR_VE = BAR_VF + NS, BAR_S = BAR_VE + NS, BAR_P = BAR_S + 2,
-                       BAR_O = BAR_P + 2, BAR_FIN = BAR_O + 2, NBARS = BAR_FIN + 1;
+  // mbarriers: Q full / free, K full/empty[NS], V full/empty[NS], and per
+  // query tile s_full, p_full, o_done, o_free (O read out); fin
+  static constexpr int BAR_QF = 0, BAR_QFREE = 1, BAR_KF = 2, BAR_KE = BAR_KF + NS,
+                       BAR_VF = BAR_KE + NS, BAR_VE = BAR_VF + NS, BAR_S = BAR_VE + NS,
+                       BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_OFREE = BAR_O + 2,
+                       BAR_FIN = BAR_OFREE + 2, NBARS = BAR_FIN + 1;
   static constexpr int OFF_SLOT = OFF_BAR + NBARS * 8;  // TMEM address, abort flag
   // + 1 KB so the swizzled tiles can start on a 1024-byte boundary
   static constexpr size_t SMEM = OFF_SLOT + 16 + 1024;
@@ -232,6 +236,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 3-D tiled tensor copy global -> shared (no multicast); x innermost.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -285,10 +299,20 @@ constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
 
 // tm_k, tm_v: K and V pools viewed as [num_blocks * heads * 16 rows][head_dim],
 // box {64, 16} (one physical block, one 64-wide slice), 128-byte swizzle.
+// tm_q: q as [tokens][query heads][head_dim], box {64, 1, 128} (128 query
+// rows of one head, one 64-wide slice), 128-byte swizzle.
+//
+// The CTAs walk the work items (query head, sequence, 256-query pair) in
+// heaviest-first order, in boustrophedon rounds: persistent (one CTA per SM)
+// for fp16, one item per CTA for bf16 (the launch decides).  The K/V rings,
+// the TMEM allocation and the barriers live across items: the loader fetches
+// the next item's Q as soon as the current item's last S products are done,
+// and a softmax group's epilogue overlaps the next item's first products.
 template <typename T, int D>
 __global__ void __launch_bounds__(384, 1)
     paged_prefill_kernel(PrefillArgs a, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v) {
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_q) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   using Cfg = PrefillConfig<D, kSplitP<T>>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, KB = Cfg::KB, NS = Cfg::NS;
@@ -298,32 +322,52 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ __align__(1024) uint8_t prefill_smem[];
   uint8_t* smem = prefill_smem + ((1024u - (smem_addr(prefill_smem) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
-
-  // grid (query head, sequence, query pair) with the pair slowest: CTAs start
-  // in linear order, so every sequence's and head's latest pairs (most keys)
-  // go first and the lightest fill the last wave
-  const int hq = blockIdx.x, s = blockIdx.y, qt = a.q_pairs - 1 - (int)blockIdx.z;
-  const int q0 = a.query_start[s];
-  const int n = a.query_start[s + 1] - q0;
-  // rows outside q / out, or beyond the launch's bound: skipped whole, reported once
-  if (n > a.max_new_tokens || (n > 0 && (q0 < 0 || q0 > a.num_tokens - n))) {
-    if (qt == 0 && hq == 0 && threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-    return;
-  }
-  if (n <= 0 || qt * 2 * BM >= n) return;
-  const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
-  const int L = a.context_lens[s];
-  if (L < n || L > cap) {  // the new tokens must be in the cache
-    if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-    return;
-  }
-  const int G = a.q_per_kv, HQ = a.heads * G, kvh = hq / G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool has1 = qt * 2 * BM + BM < n;  // second query tile holds queries
-  // key tiles each query tile visits (up to its last query's position)
-  const int nkt0 = (L - n + min(n, qt * 2 * BM + BM) - 1 + BN) / BN;
-  const int nkt1 = has1 ? (L - n + min(n, qt * 2 * BM + 2 * BM) - 1 + BN) / BN : 0;
-  const int nkt = has1 ? nkt1 : nkt0;
+  const int G = a.q_per_kv, HQ = a.heads * G;
+  const int num_items = HQ * a.num_seqs * a.q_pairs;
+  // The CTA's k-th item: rounds of gridDim.x items, taken left to right in
+  // even rounds and right to left in odd ones, so that every CTA gets a fair
+  // share of the heavy (early) and light (late) items.
+  const int rounds = (num_items + gridDim.x - 1) / gridDim.x;
+  auto nth_item = [&](int k) {
+    return k * (int)gridDim.x + ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
+  const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
+
+  // One work item: (query head, sequence, query pair) with the pair slowest,
+  // so that every head's and sequence's latest pairs (most keys) come first.
+  struct Item {
+    int hq, s, qt, q0, n, L, kvh, nkt0, nkt1, nkt;
+    bool has1;
+  };
+  // Whether item w holds work; a sequence the launch cannot take is reported
+  // once (by its item with pair 0 and head 0) and skipped.
+  auto item_of = [&](int w, Item& it, bool report) {
+    it.hq = w % HQ;
+    it.s = (w / HQ) % a.num_seqs;
+    it.qt = a.q_pairs - 1 - w / (HQ * a.num_seqs);
+    it.q0 = a.query_start[it.s];
+    it.n = a.query_start[it.s + 1] - it.q0;
+    const bool first = it.qt == 0 && it.hq == 0;
+    // rows outside q / out, or beyond the launch's bound
+    if (it.n > a.max_new_tokens || (it.n > 0 && (it.q0 < 0 || it.q0 > a.num_tokens - it.n))) {
+      if (report && first) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+      return false;
+    }
+    if (it.n <= 0 || it.qt * 2 * BM >= it.n) return false;
+    it.L = a.context_lens[it.s];
+    if (it.L < it.n || it.L > cap) {  // the new tokens must be in the cache
+      if (report && first) atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+      return false;
+    }
+    it.kvh = it.hq / G;
+    it.has1 = it.qt * 2 * BM + BM < it.n;  // second query tile holds queries
+    // key tiles each query tile visits (up to its last query's position)
+    it.nkt0 = (it.L - it.n + min(it.n, it.qt * 2 * BM + BM) - 1 + BN) / BN;
+    it.nkt1 = it.has1 ? (it.L - it.n + min(it.n, it.qt * 2 * BM + 2 * BM) - 1 + BN) / BN : 0;
+    it.nkt = it.has1 ? it.nkt1 : it.nkt0;
+    return true;
+  };
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   auto bar = [&](int i) { return smem_addr(&bars[i]); };
@@ -338,8 +382,8 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (threadIdx.x == 32) {
-    mbar_init(bar(Cfg::BAR_Q + 0), BM / 32);  // one arrival per softmax warp
-    mbar_init(bar(Cfg::BAR_Q + 1), BM / 32);
+    mbar_init(bar(Cfg::BAR_QF), 1);
+    mbar_init(bar(Cfg::BAR_QFREE), 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(bar(Cfg::BAR_KF + i), 1);
       mbar_init(bar(Cfg::BAR_KE + i), 1);
@@ -348,8 +392,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Cfg::BAR_S + w), 1);
-      mbar_init(bar(Cfg::BAR_P + w), BM / 32);
+      mbar_init(bar(Cfg::BAR_P + w), BM / 32);  // one arrival per softmax warp
       mbar_init(bar(Cfg::BAR_O + w), 1);
+      mbar_init(bar(Cfg::BAR_OFREE + w), BM / 32);
     }
     mbar_init(bar(Cfg::BAR_FIN), 1);
     *abort_flag = 0;
@@ -372,93 +417,120 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 8) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Cfg::REGS_OTHER));
   if (warp == Cfg::LOAD_WARP) {
-    // ---- loader: K and V of key tile j into stage j % NS of their rings ----------
+    // ---- loader: Q of each item, then K and V of key tile j into the next
+    // stage of their rings (positions counted across items) ----------------------
     // K runs one tile ahead of V: a K stage frees once both S products of its
     // tile are issued, a V stage only after both P.V products.
-    const int32_t* table = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-    int k_issued = 0, v_issued = 0;
-    // lane i < blocks in tile j: that block's id (fetched by all lanes at once)
-    auto tile_blocks = [&](int j, int& nblk, int& valid) {
-      valid = min(BN, L - j * BN);
-      nblk = (valid + kBlock - 1) / kBlock;
-      int32_t blk = 0;
-      if (lane < nblk) {
-        blk = table[j * (BN / kBlock) + lane];
-        if (blk < 0 || blk >= a.num_blocks) {
-          atomicOr(a.err, PA_DEVERR_BLOCK_ID);
-          blk = 0;
+    uint32_t kc = 0, vc = 0;  // K / V fills issued
+    int items = 0;            // items whose Q was loaded
+    bool ok = true;
+    for (int k = 0; ok && k < rounds; ++k) {
+      const int w = nth_item(k);
+      Item it;
+      if (w >= num_items || !item_of(w, it, false)) continue;
+      const int32_t* table = a.block_tables + (int64_t)it.s * a.max_blocks_per_seq;
+      // lane i < blocks in tile j: that block's id (fetched by all lanes at once)
+      auto tile_blocks = [&](int j, int& nblk, int& valid) {
+        valid = min(BN, it.L - j * BN);
+        nblk = (valid + kBlock - 1) / kBlock;
+        int32_t blk = 0;
+        if (lane < nblk) {
+          blk = table[j * (BN / kBlock) + lane];
+          if (blk < 0 || blk >= a.num_blocks) {
+            atomicOr(a.err, PA_DEVERR_BLOCK_ID);
+            blk = 0;
+          }
         }
-      }
-      return blk;
-    };
-    auto load_k = [&](int j) {
-      int nblk, valid;
-      const int32_t blk = tile_blocks(j, nblk, valid);
-      const int st = j % NS;
-      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_KE + st), ((j / NS) - 1) & 1, abort_flag))
-        return false;
-      if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_KF + st), (uint32_t)nblk * KB * kBlock * 128);
-      __syncwarp();
-      if (lane < nblk) {  // K rows past the context are masked out of S by selection
-        const int row0 = (int)(((int64_t)blk * a.heads + kvh) * kBlock);
+        return blk;
+      };
+      auto load_k = [&](int j) {
+        int nblk, valid;
+        const int32_t blk = tile_blocks(j, nblk, valid);
+        const int st = kc % NS;
+        if (kc >= NS && !warp_wait_or_abort(bar(Cfg::BAR_KE + st), ((kc / NS) - 1) & 1, abort_flag))
+          return false;
+        if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_KF + st), (uint32_t)nblk * KB * kBlock * 128);
+        __syncwarp();
+        if (lane < nblk) {  // K rows past the context are masked out of S by selection
+          const int row0 = (int)(((int64_t)blk * a.heads + it.kvh) * kBlock);
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(sbase + Cfg::OFF_K + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
-                      &tm_k, kb * 64, row0, bar(Cfg::BAR_KF + st));
-      }
-      k_issued = j + 1;
-      return true;
-    };
-    auto load_v = [&](int j) {
-      int nblk, valid;
-      const int32_t blk = tile_blocks(j, nblk, valid);
-      const int st = j % NS;
-      if (j >= NS && !warp_wait_or_abort(bar(Cfg::BAR_VE + st), ((j / NS) - 1) & 1, abort_flag))
-        return false;
-      // V rows at or past the context are zeroed (their weights are zero, but
-      // stale bits may be NaN).  A partly filled last block's valid rows are
-      // copied by the lanes, so every tensor copy moves a whole block.
-      const bool partial = valid < nblk * kBlock;
-      const int32_t last_blk = __shfl_sync(kFullMask, blk, nblk - 1);
-      uint8_t* gV = smem + Cfg::OFF_V + st * Cfg::KV_BYTES;
-      if (valid < BN) {
-        const int r_lo = partial ? (nblk - 1) * kBlock : valid;
-        const T* src = static_cast<const T*>(a.v_pool) +
-                       (((int64_t)last_blk * a.heads + kvh) * kBlock) * D;
-        for (int idx = lane; idx < (BN - r_lo) * KB * 8; idx += 32) {
-          const int r = r_lo + idx / (KB * 8), c = idx % (KB * 8);
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (r < valid) v = *reinterpret_cast<const uint4*>(src + (int64_t)(r - r_lo) * D + c * 8);
-          *reinterpret_cast<uint4*>(gV + (c >> 3) * (BN * 128) + sw128_off(r, c & 7)) = v;
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sbase + Cfg::OFF_K + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
+                        &tm_k, kb * 64, row0, bar(Cfg::BAR_KF + st));
         }
-        fence_proxy_async_shared();
-      }
-      const int nfull = partial ? nblk - 1 : nblk;
-      __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_VF + st), (uint32_t)nfull * KB * kBlock * 128);
-      __syncwarp();
-      if (lane < nfull) {
-        const int row0 = (int)(((int64_t)blk * a.heads + kvh) * kBlock);
+        ++kc;
+        return true;
+      };
+      auto load_v = [&](int j) {
+        int nblk, valid;
+        const int32_t blk = tile_blocks(j, nblk, valid);
+        const int st = vc % NS;
+        if (vc >= NS && !warp_wait_or_abort(bar(Cfg::BAR_VE + st), ((vc / NS) - 1) & 1, abort_flag))
+          return false;
+        // V rows at or past the context are zeroed (their weights are zero, but
+        // stale bits may be NaN).  A partly filled last block's valid rows are
+        // copied by the lanes, so every tensor copy moves a whole block.
+        const bool partial = valid < nblk * kBlock;
+        const int32_t last_blk = __shfl_sync(kFullMask, blk, nblk - 1);
+        uint8_t* gV = smem + Cfg::OFF_V + st * Cfg::KV_BYTES;
+        if (valid < BN) {
+          const int r_lo = partial ? (nblk - 1) * kBlock : valid;
+          const T* src = static_cast<const T*>(a.v_pool) +
+                         (((int64_t)last_blk * a.heads + it.kvh) * kBlock) * D;
+          for (int idx = lane; idx < (BN - r_lo) * KB * 8; idx += 32) {
+            const int r = r_lo + idx / (KB * 8), c = idx % (KB * 8);
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r < valid) v = *reinterpret_cast<const uint4*>(src + (int64_t)(r - r_lo) * D + c * 8);
+            *reinterpret_cast<uint4*>(gV + (c >> 3) * (BN * 128) + sw128_off(r, c & 7)) = v;
+          }
+          fence_proxy_async_shared();
+        }
+        const int nfull = partial ? nblk - 1 : nblk;
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(bar(Cfg::BAR_VF + st), (uint32_t)nfull * KB * kBlock * 128);
+        __syncwarp();
+        if (lane < nfull) {
+          const int row0 = (int)(((int64_t)blk * a.heads + it.kvh) * kBlock);
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(sbase + Cfg::OFF_V + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
-                      &tm_v, kb * 64, row0, bar(Cfg::BAR_VF + st));
-      }
-      v_issued = j + 1;
-      return true;
-    };
-    for (int t = 0; t <= nkt; ++t) {
-      if ((t < nkt && !load_k(t)) || (t >= 1 && !load_v(t - 1))) {
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sbase + Cfg::OFF_V + st * Cfg::KV_BYTES + kb * (BN * 128) + lane * (kBlock * 128),
+                        &tm_v, kb * 64, row0, bar(Cfg::BAR_VF + st));
+        }
+        ++vc;
+        return true;
+      };
+      // Q of the item's query tiles, once the previous item's S products are
+      // done with the Q buffers (rows past the tokens come in as zeros)
+      if (items > 0 && !warp_wait_or_abort(bar(Cfg::BAR_QFREE), (items - 1) & 1, abort_flag)) {
         give_up();
         break;
       }
+      if (lane == 0) {
+        const int tiles = it.has1 ? 2 : 1;
+        mbar_arrive_expect_tx(bar(Cfg::BAR_QF), (uint32_t)tiles * Cfg::Q_BYTES);
+        for (int t = 0; t < tiles; ++t)
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(sbase + Cfg::OFF_Q + t * Cfg::Q_BYTES + kb * (BM * 128), &tm_q, kb * 64,
+                        it.hq, it.q0 + it.qt * 2 * BM + t * BM, bar(Cfg::BAR_QF));
+      }
+      __syncwarp();
+      ++items;
+      for (int t = 0; t <= it.nkt; ++t) {
+        if ((t < it.nkt && !load_k(t)) || (t >= 1 && !load_v(t - 1))) {
+          give_up();
+          ok = false;
+          break;
+        }
+      }
     }
-    // let the copies of the last stages land before the CTA releases its memory
+    // let the last copies land before the CTA releases its memory
     if (lane == 0) {
-      for (int j = max(0, k_issued - NS); j < k_issued; ++j)
+      for (uint32_t j = kc > NS ? kc - NS : 0; j < kc; ++j)
         mbar_wait_bounded(bar(Cfg::BAR_KF + j % NS), (j / NS) & 1);
-      for (int j = max(0, v_issued - NS); j < v_issued; ++j)
+      for (uint32_t j = vc > NS ? vc - NS : 0; j < vc; ++j)
         mbar_wait_bounded(bar(Cfg::BAR_VF + j % NS), (j / NS) & 1);
+      if (items > 0) mbar_wait_bounded(bar(Cfg::BAR_QF), (items - 1) & 1);
     }
   } else if (warp == Cfg::MMA_WARP) {
     // ---- MMA issue ------------------------------------------------------------------
@@ -494,49 +566,71 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr (kSplitP<T>) umma_f16_ts(od, pa + Cfg::P_LO + kk * 8, bd, IDESC_PV, 1u);
         }
       };
-      int k_ready = -1, v_ready = -1;  // last tiles whose K / V stage was seen full
-      auto wait_full = [&](int base, int j, int& ready) {
-        if (j <= ready) return true;
-        if (!mbar_wait_or_abort(bar(base + j % NS), (j / NS) & 1, abort_flag)) return false;
-        ready = j;
+      // ring positions (counted across items) whose K / V stage was seen full
+      int64_t k_ready = -1, v_ready = -1;
+      auto wait_full = [&](int base, uint32_t pos, int64_t& ready) {
+        if ((int64_t)pos <= ready) return true;
+        if (!mbar_wait_or_abort(bar(base + pos % NS), (pos / NS) & 1, abort_flag)) return false;
+        ready = pos;
         tc_fence_after();
         return true;
       };
-      bool ok = mbar_wait_or_abort(bar(Cfg::BAR_Q + 0), 0, abort_flag) &&
-                wait_full(Cfg::BAR_KF, 0, k_ready) &&
-                (!has1 || mbar_wait_or_abort(bar(Cfg::BAR_Q + 1), 0, abort_flag));
-      if (ok) {
+      uint32_t kc = 0, vc = 0;    // K / V tiles consumed
+      int items = 0;              // items started
+      int pc[2] = {0, 0};         // p_full phases consumed, per query tile
+      int ow[2] = {0, 0};         // items in which each query tile had work
+      bool ok = true;
+      for (int k = 0; ok && k < rounds; ++k) {
+        const int w = nth_item(k);
+        Item it;
+        if (w >= num_items || !item_of(w, it, false)) continue;
+        const int nkt = it.nkt;
+        ok = mbar_wait_or_abort(bar(Cfg::BAR_QF), items & 1, abort_flag) &&
+             wait_full(Cfg::BAR_KF, kc, k_ready);
+        if (!ok) break;
+        ++items;
         tc_fence_after();
-        issue_s(0, 0);
+        issue_s(0, kc % NS);
         umma_commit(bar(Cfg::BAR_S + 0));
-        if (has1) {
-          issue_s(1, 0);
+        if (it.has1) {
+          issue_s(1, kc % NS);
           umma_commit(bar(Cfg::BAR_S + 1));
         }
-        umma_commit(bar(Cfg::BAR_KE + 0));
-      }
-      for (int j = 0; ok && j < nkt; ++j) {
+        umma_commit(bar(Cfg::BAR_KE + kc % NS));
+        if (nkt == 1) umma_commit(bar(Cfg::BAR_QFREE));  // Q is no longer read
+        for (int j = 0; ok && j < nkt; ++j) {
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const int nk = w == 0 ? nkt0 : nkt1;
-          if (j >= nk) continue;
-          if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + w), j & 1, abort_flag) &&
-                     wait_full(Cfg::BAR_VF, j, v_ready)))
-            break;
-          tc_fence_after();
-          issue_pv(w, j % NS, j == 0);
-          if (j == nk - 1) {
-            umma_commit(bar(Cfg::BAR_O + w));
-          } else {
-            if (!(ok = wait_full(Cfg::BAR_KF, j + 1, k_ready))) break;
-            issue_s(w, (j + 1) % NS);
-            umma_commit(bar(Cfg::BAR_S + w));
+          for (int t = 0; t < 2; ++t) {
+            const int nk = t == 0 ? it.nkt0 : it.nkt1;
+            if (j >= nk) continue;
+            if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + t), pc[t] & 1, abort_flag) &&
+                       wait_full(Cfg::BAR_VF, vc + j, v_ready)))
+              break;
+            ++pc[t];
+            // the first P.V of an item overwrites O: its last reader must be done
+            if (j == 0 && ow[t] > 0 &&
+                !(ok = mbar_wait_or_abort(bar(Cfg::BAR_OFREE + t), (ow[t] - 1) & 1, abort_flag)))
+              break;
+            tc_fence_after();
+            issue_pv(t, (vc + j) % NS, j == 0);
+            if (j == nk - 1) {
+              umma_commit(bar(Cfg::BAR_O + t));
+            } else {
+              if (!(ok = wait_full(Cfg::BAR_KF, kc + j + 1, k_ready))) break;
+              issue_s(t, (kc + j + 1) % NS);
+              umma_commit(bar(Cfg::BAR_S + t));
+            }
+          }
+          if (ok) {
+            umma_commit(bar(Cfg::BAR_VE + (vc + j) % NS));
+            if (j + 1 < nkt) umma_commit(bar(Cfg::BAR_KE + (kc + j + 1) % NS));
+            if (j + 2 == nkt) umma_commit(bar(Cfg::BAR_QFREE));  // the item's last S are issued
           }
         }
-        if (ok) {
-          umma_commit(bar(Cfg::BAR_VE + j % NS));
-          if (j + 1 < nkt) umma_commit(bar(Cfg::BAR_KE + (j + 1) % NS));
-        }
+        kc += nkt;
+        vc += nkt;
+        ow[0] += it.nkt0 > 0;
+        ow[1] += it.nkt1 > 0;
       }
       if (!ok) give_up();
       // every product issued has completed before TMEM and shared memory go
@@ -549,39 +643,27 @@ __global__ void __launch_bounds__(384, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Cfg::REGS_SOFTMAX));
     // ---- softmax warpgroups -----------------------------------------------------------
     const int w = warp >> 2, r = threadIdx.x & (BM - 1);
-    const int qbase = qt * 2 * BM + w * BM;
-    const int nk = w == 0 ? nkt0 : nkt1;
-    if (qbase < n) {
-      // Q tile: row rr = query qbase + rr, zero past the new tokens
-      uint8_t* sQ = smem + Cfg::OFF_Q + w * Cfg::Q_BYTES;
-      constexpr int CH = D / 8;
-      for (int idx = r; idx < BM * CH; idx += BM) {
-        const int rr = idx / CH, c = idx % CH;
-        uint8_t* dst = sQ + (c >> 3) * (BM * 128) + sw128_off(rr, c & 7);
-        if (qbase + rr < n)
-          cp_async16(smem_addr(dst),
-                     static_cast<const T*>(a.q) + ((int64_t)(q0 + qbase + rr) * HQ + hq) * D + c * 8);
-        else
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(Cfg::BAR_Q + w));
-
+    const float sl2 = a.scale_log2;
+    const float masked_raw = sl2 >= 0.f ? -INFINITY : INFINITY;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + Cfg::S_COL0 + w * BN;
+    const uint32_t o_addr = tmem + lane_base + Cfg::O_COL0 + w * D;
+    int sc_ph = 0, oc_ph = 0;  // s_full / o_done phases consumed (across items)
+    bool ok = true;
+    for (int k = 0; ok && k < rounds; ++k) {
+      const int wi = nth_item(k);
+      Item it;
+      if (wi >= num_items || !item_of(wi, it, threadIdx.x == 0)) continue;
+      const int qbase = it.qt * 2 * BM + w * BM;
+      const int nk = w == 0 ? it.nkt0 : it.nkt1;
+      if (nk == 0) continue;  // this query tile of the item holds no queries
       const int qi = qbase + r;
-      const bool row_valid = qi < n;
-      const int pos = L - n + qi;  // this query's position
-      const float sl2 = a.scale_log2;
-      const float masked_raw = sl2 >= 0.f ? -INFINITY : INFINITY;
-      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + Cfg::S_COL0 + w * BN;
-      const uint32_t o_addr = tmem + lane_base + Cfg::O_COL0 + w * D;
+      const bool row_valid = qi < it.n;
+      const int pos = it.L - it.n + qi;  // this query's position
       float m_used = -INFINITY, l_run = 0.f;
-      bool ok = true;
       for (int j = 0; j < nk; ++j) {
-        if (!(ok = warp_wait_or_abort(bar(Cfg::BAR_S + w), j & 1, abort_flag))) break;
+        if (!(ok = warp_wait_or_abort(bar(Cfg::BAR_S + w), sc_ph & 1, abort_flag))) break;
+        ++sc_ph;
         tc_fence_after();
         float2 sv[BN / 2];
         float* sc = reinterpret_cast<float*>(sv);
@@ -699,32 +781,34 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(Cfg::BAR_P + w));
       }
-      if (ok) ok = warp_wait_or_abort(bar(Cfg::BAR_O + w), 0, abort_flag);
-      if (!ok) {
-        give_up();
-      } else {
-        tc_fence_after();
-        // ---- O / l for this row -----------------------------------------------------
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        T* dst = static_cast<T*>(a.out) + ((int64_t)(q0 + qi) * HQ + hq) * D;
+      if (ok) ok = warp_wait_or_abort(bar(Cfg::BAR_O + w), oc_ph & 1, abort_flag);
+      if (!ok) break;
+      ++oc_ph;
+      tc_fence_after();
+      // ---- O / l for this row, then O is free for the next item -------------------------
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      T* dst = static_cast<T*>(a.out) + ((int64_t)(it.q0 + qi) * HQ + it.hq) * D;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tmem_ld32(o_addr + c0, o);
-          if (row_valid) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        tmem_ld32(o_addr + c0, o);
+        if (row_valid) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 v;
-              v.x = MmaType<T>::pack(o[i] * inv, o[i + 1] * inv);
-              v.y = MmaType<T>::pack(o[i + 2] * inv, o[i + 3] * inv);
-              v.z = MmaType<T>::pack(o[i + 4] * inv, o[i + 5] * inv);
-              v.w = MmaType<T>::pack(o[i + 6] * inv, o[i + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + c0 + i) = v;
-            }
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = MmaType<T>::pack(o[i] * inv, o[i + 1] * inv);
+            v.y = MmaType<T>::pack(o[i + 2] * inv, o[i + 3] * inv);
+            v.z = MmaType<T>::pack(o[i + 4] * inv, o[i + 5] * inv);
+            v.w = MmaType<T>::pack(o[i + 6] * inv, o[i + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c0 + i) = v;
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(Cfg::BAR_OFREE + w));
     }
+    if (!ok) give_up();
   }
   // every role is done and every copy or product it issued has landed
   tc_fence_before();
