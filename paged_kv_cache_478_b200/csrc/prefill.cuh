@@ -80,6 +80,13 @@ struct PrefillConfig {
   static constexpr int BN = 128;        // keys per tile
   static constexpr int KB = D / 64;     // 128-byte K-blocks across head_dim
   static constexpr int NS = D == 128 ? 2 : 3;  // stages of the K ring and of the V ring
+#ifndef PA_PREFILL_P_CHUNKS
+#define PA_PREFILL_P_CHUNKS 2
+#endif
+  // P goes to the tensor core in PC pieces of BN / PC keys, each handed over
+  // as soon as it is in TMEM
+  static constexpr int PC = PA_PREFILL_P_CHUNKS;
+  static_assert(PC == 1 || PC == 2 || PC == 4, "P pieces");
   static constexpr int LOAD_WARP = 8, MMA_WARP = 9;  // warps 10-11 only fill the warpgroup
   static constexpr int THREADS = 384;
   // Launched at 168 registers a thread (384 x 168 fit the register file);
@@ -95,11 +102,12 @@ struct PrefillConfig {
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;           // [stage]
   static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
   // mbarriers: Q full / free, K full/empty[NS], V full/empty[NS], and per
-  // query tile s_full, p_full, o_done, o_free (O read out); fin
+  // query tile s_full, p_full of each P piece (BAR_P + 2 * piece + tile),
+  // o_done, o_free (O read out); fin
   static constexpr int BAR_QF = 0, BAR_QFREE = 1, BAR_KF = 2, BAR_KE = BAR_KF + NS,
                        BAR_VF = BAR_KE + NS, BAR_VE = BAR_VF + NS, BAR_S = BAR_VE + NS,
-                       BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_OFREE = BAR_O + 2,
-                       BAR_FIN = BAR_OFREE + 2, NBARS = BAR_FIN + 1;
+                       BAR_P = BAR_S + 2, BAR_O = BAR_P + 2 * PC,
+                       BAR_OFREE = BAR_O + 2, BAR_FIN = BAR_OFREE + 2, NBARS = BAR_FIN + 1;
   static constexpr int OFF_SLOT = OFF_BAR + NBARS * 8;  // TMEM address, abort flag
   // + 1 KB so the swizzled tiles can start on a 1024-byte boundary
   static constexpr size_t SMEM = OFF_SLOT + 16 + 1024;
@@ -392,7 +400,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(Cfg::BAR_S + w), 1);
-      mbar_init(bar(Cfg::BAR_P + w), BM / 32);  // one arrival per softmax warp
+      for (int c = 0; c < Cfg::PC; ++c)
+        mbar_init(bar(Cfg::BAR_P + 2 * c + w), BM / 32);  // one arrival per softmax warp
       mbar_init(bar(Cfg::BAR_O + w), 1);
       mbar_init(bar(Cfg::BAR_OFREE + w), BM / 32);
     }
@@ -554,12 +563,13 @@ __global__ void __launch_bounds__(384, 1)
           umma_f16(sd, at(qd, kofs), at(kd, kofs_b), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int w, int st, bool first) {
+      // P.V over the keys of P piece c of a tile
+      auto issue_pv = [&](int w, int st, bool first, int c) {
         const uint32_t pa = tmem + Cfg::S_COL0 + w * BN;  // P over S, 8 columns per 16 keys
         const uint32_t od = tmem + Cfg::O_COL0 + w * D;
         const uint64_t vd = at(dv, st * Cfg::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int kk = c * (BN / 16 / Cfg::PC); kk < (c + 1) * (BN / 16 / Cfg::PC); ++kk) {
           // V is MN-major: 64-dim blocks LBO apart, 8-key groups 1024 bytes apart
           const uint64_t bd = at(vd, kk * 2048);
           umma_f16_ts(od, pa + kk * 8, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
@@ -603,7 +613,8 @@ __global__ void __launch_bounds__(384, 1)
           for (int t = 0; t < 2; ++t) {
             const int nk = t == 0 ? it.nkt0 : it.nkt1;
             if (j >= nk) continue;
-            if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + t), pc[t] & 1, abort_flag) &&
+            const uint32_t ph = pc[t] & 1;
+            if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + t), ph, abort_flag) &&
                        wait_full(Cfg::BAR_VF, vc + j, v_ready)))
               break;
             ++pc[t];
@@ -612,7 +623,15 @@ __global__ void __launch_bounds__(384, 1)
                 !(ok = mbar_wait_or_abort(bar(Cfg::BAR_OFREE + t), (ow[t] - 1) & 1, abort_flag)))
               break;
             tc_fence_after();
-            issue_pv(t, (vc + j) % NS, j == 0);
+            // P.V of each piece runs while the softmax finishes the next ones
+            issue_pv(t, (vc + j) % NS, j == 0, 0);
+#pragma unroll
+            for (int c = 1; c < Cfg::PC; ++c) {
+              if (!(ok = mbar_wait_or_abort(bar(Cfg::BAR_P + 2 * c + t), ph, abort_flag))) break;
+              tc_fence_after();
+              issue_pv(t, (vc + j) % NS, j == 0, c);
+            }
+            if (!ok) break;
             if (j == nk - 1) {
               umma_commit(bar(Cfg::BAR_O + t));
             } else {
@@ -685,10 +704,11 @@ __global__ void __launch_bounds__(384, 1)
         // split keeps the ALU busiest, and -1 % for fp16, which finds the max
         // first.
         const float2 sl2v = make_float2(sl2, sl2);
-        auto weights = [&](float mb) {
+        // weights of the keys [2 * i0, 2 * i1) against the reference max mb
+        auto weights = [&](float mb, int i0, int i1) {
           const float2 nmb = make_float2(-mb, -mb);
 #pragma unroll
-          for (int i = 0; i < BN / 2; ++i) {
+          for (int i = i0; i < i1; ++i) {
             const float2 x = __ffma2_rn(sv[i], sl2v, nmb);
             sv[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           }
@@ -705,7 +725,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 8; c < BN; c += 2) mx8[(c >> 1) & 7] = fmin3f(mx8[(c >> 1) & 7], sc[c], sc[c + 1]);
         }
-        if (ahead) weights(m_used);  // independent of the max: overlaps it
+        if (ahead) weights(m_used, 0, BN / 2);  // independent of the max: overlaps it
 #pragma unroll
         for (int i = 4; i >= 1; i >>= 1)
 #pragma unroll
@@ -714,8 +734,10 @@ __global__ void __launch_bounds__(384, 1)
         const float m_tile = sl2 == 0.f ? 0.f : mx8[0] * sl2;
         // move the reference max only when a weight would exceed 2^8
         const bool move = m_tile > m_used + 8.f;
+        const bool any_move = __any_sync(kFullMask, move);
         float alpha = 1.f;
-        if (__any_sync(kFullMask, move) || !ahead) {
+        bool have_w = ahead;  // the weights above stand unless the reference moves
+        if (any_move || !ahead) {
           if (move) {
             alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - m_tile);
             m_used = m_tile;
@@ -730,24 +752,14 @@ __global__ void __launch_bounds__(384, 1)
                 if (!row_valid || j * BN + c > pos) sc[c] = masked_raw;
             }
           }
-          weights(m_used == -INFINITY ? 0.f : m_used);
+          have_w = false;
         }
-        if (need_mask) {  // a zero scale keeps masked scores finite: select them out
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (!row_valid || j * BN + c > pos) sc[c] = 0.f;
-        }
-        float2 sum4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sum4[i] = sv[i];
-#pragma unroll
-        for (int i = 4; i < BN / 2; ++i) sum4[i & 3] = __fadd2_rn(sum4[i & 3], sv[i]);
-        sum4[0] = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
-        l_run = fmaf(l_run, alpha, sum4[0].x + sum4[0].y);
-        // rescale this row of O (P.V of tile j-1 has completed: the product
-        // S of tile j was committed after it)
+        const float mb = m_used == -INFINITY ? 0.f : m_used;
+        // rescale this row of O before any P.V of this tile lands in it (P.V
+        // of tile j-1 has completed: the product S of tile j was committed
+        // after it)
         __syncwarp();
-        if (j > 0 && __any_sync(kFullMask, move)) {
+        if (j > 0 && any_move) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             float o[32];
@@ -757,29 +769,49 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(o_addr + c0, o);
           }
         }
-        // this row of P over S in TMEM: column c holds keys 2c (low half) and
-        // 2c + 1; the S values were all read above
+        // this row of P over S in TMEM, in PC pieces of BN/PC keys, each
+        // handed to the MMA warp as soon as it is stored, so that P.V of one
+        // piece runs while the next is computed.  Column c holds keys 2c (low
+        // half) and 2c + 1; the S values were all read above.
+        constexpr int PK = BN / Cfg::PC;  // keys per piece
 #pragma unroll
-        for (int h = 0; h < BN / 32; ++h) {
-          if constexpr (kSplitP<T>) {
-            uint32_t hi[16], lo[16];
+        for (int pi = 0; pi < Cfg::PC; ++pi) {
+          if (!have_w) weights(mb, pi * (PK / 2), (pi + 1) * (PK / 2));
+          if (need_mask) {  // a zero scale keeps masked scores finite: select them out
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pack_split<T>(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1], hi[i], lo[i]);
-            tmem_st16_nowait(s_addr + Cfg::P_LO + 16 * h, lo);
-            tmem_st16_nowait(s_addr + 16 * h, hi);
-          } else {
-            uint32_t hi[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              hi[i] = MmaType<T>::pack(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1]);
-            tmem_st16_nowait(s_addr + 16 * h, hi);
+            for (int c = pi * PK; c < (pi + 1) * PK; ++c)
+              if (!row_valid || j * BN + c > pos) sc[c] = 0.f;
           }
+#pragma unroll
+          for (int h = pi * (PK / 32); h < (pi + 1) * (PK / 32); ++h) {
+            if constexpr (kSplitP<T>) {
+              uint32_t hi[16], lo[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pack_split<T>(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1], hi[i], lo[i]);
+              tmem_st16_nowait(s_addr + Cfg::P_LO + 16 * h, lo);
+              tmem_st16_nowait(s_addr + 16 * h, hi);
+            } else {
+              uint32_t hi[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                hi[i] = MmaType<T>::pack(sc[32 * h + 2 * i], sc[32 * h + 2 * i + 1]);
+              tmem_st16_nowait(s_addr + 16 * h, hi);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(Cfg::BAR_P + 2 * pi + w));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(Cfg::BAR_P + w));
+        // the row sum, off the path to P.V
+        float2 sum4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum4[i] = sv[i];
+#pragma unroll
+        for (int i = 4; i < BN / 2; ++i) sum4[i & 3] = __fadd2_rn(sum4[i & 3], sv[i]);
+        sum4[0] = __fadd2_rn(__fadd2_rn(sum4[0], sum4[1]), __fadd2_rn(sum4[2], sum4[3]));
+        l_run = fmaf(l_run, alpha, sum4[0].x + sum4[0].y);
       }
       if (ok) ok = warp_wait_or_abort(bar(Cfg::BAR_O + w), oc_ph & 1, abort_flag);
       if (!ok) break;
