@@ -115,7 +115,10 @@ int rings_for(int G) { return warps_for(G) / G; }
 // kernel (one warp per KV head); MHA, pairs (measured faster on CUDA cores)
 // and fp32 pools take the CUDA-core kernel.
 bool use_gqa_mma(const pa_pool* pool) { return pool->q_per_kv >= 4 && pool->dtype != PA_F32; }
-constexpr int kGqaStages = 2;
+#ifndef PA_GQA_STAGES
+#define PA_GQA_STAGES 2
+#endif
+constexpr int kGqaStages = PA_GQA_STAGES;  // per-warp ring depth of the tensor-core kernel
 
 int kv_heads_per_item(const pa_pool* pool) {
   return use_gqa_mma(pool) ? GqaConfig<__half, 128, kGqaStages>::WARPS : rings_for(pool->q_per_kv);
