@@ -30,9 +30,14 @@
 
 namespace pa {
 
+#ifndef PA_GQA_WARPS
+#define PA_GQA_WARPS 4
+#endif
+
 template <typename T, int D, int NSTAGE>
 struct GqaConfig {
-  static constexpr int WARPS = 4;            // KV heads per work item, one per warp
+  static constexpr int WARPS = PA_GQA_WARPS;  // KV heads per work item, one per warp
+  static_assert(WARPS >= 1 && WARPS <= 4, "warps per CTA");
   static constexpr int THREADS = WARPS * 32;
   static constexpr int ROW_BYTES = D * 2;
   static constexpr int PITCH = ROW_BYTES + 16;
