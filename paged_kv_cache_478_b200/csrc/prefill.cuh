@@ -87,6 +87,9 @@ struct PrefillConfig {
   // as soon as it is in TMEM
   static constexpr int PC = PA_PREFILL_P_CHUNKS;
   static_assert(PC == 1 || PC == 2 || PC == 4, "P pieces");
+  // keys [piece_begin(c), piece_end(c)) form P piece c
+  static constexpr int piece_begin(int c) { return c * (BN / PC); }
+  static constexpr int piece_end(int c) { return (c + 1) * (BN / PC); }
   static constexpr int LOAD_WARP = 8, MMA_WARP = 9;  // warps 10-11 only fill the warpgroup
   static constexpr int THREADS = 384;
   // Launched at 168 registers a thread (384 x 168 fit the register file);
@@ -569,7 +572,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t od = tmem + Cfg::O_COL0 + w * D;
         const uint64_t vd = at(dv, st * Cfg::KV_BYTES);
 #pragma unroll
-        for (int kk = c * (BN / 16 / Cfg::PC); kk < (c + 1) * (BN / 16 / Cfg::PC); ++kk) {
+        for (int kk = Cfg::piece_begin(c) / 16; kk < Cfg::piece_end(c) / 16; ++kk) {
           // V is MN-major: 64-dim blocks LBO apart, 8-key groups 1024 bytes apart
           const uint64_t bd = at(vd, kk * 2048);
           umma_f16_ts(od, pa + kk * 8, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
@@ -773,17 +776,19 @@ __global__ void __launch_bounds__(384, 1)
         // handed to the MMA warp as soon as it is stored, so that P.V of one
         // piece runs while the next is computed.  Column c holds keys 2c (low
         // half) and 2c + 1; the S values were all read above.
-        constexpr int PK = BN / Cfg::PC;  // keys per piece
-#pragma unroll
-        for (int pi = 0; pi < Cfg::PC; ++pi) {
-          if (!have_w) weights(mb, pi * (PK / 2), (pi + 1) * (PK / 2));
+        // the piece index is a compile-time constant, so every index into sc
+        // is one and the row stays in registers
+        auto piece = [&](auto pc_const) {
+          constexpr int pi = decltype(pc_const)::value;
+          constexpr int k0 = Cfg::piece_begin(pi), k1 = Cfg::piece_end(pi);
+          if (!have_w) weights(mb, k0 / 2, k1 / 2);
           if (need_mask) {  // a zero scale keeps masked scores finite: select them out
 #pragma unroll
-            for (int c = pi * PK; c < (pi + 1) * PK; ++c)
+            for (int c = k0; c < k1; ++c)
               if (!row_valid || j * BN + c > pos) sc[c] = 0.f;
           }
 #pragma unroll
-          for (int h = pi * (PK / 32); h < (pi + 1) * (PK / 32); ++h) {
+          for (int h = k0 / 32; h < k1 / 32; ++h) {
             if constexpr (kSplitP<T>) {
               uint32_t hi[16], lo[16];
 #pragma unroll
@@ -803,6 +808,12 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(Cfg::BAR_P + 2 * pi + w));
+        };
+        piece(std::integral_constant<int, 0>{});
+        if constexpr (Cfg::PC > 1) piece(std::integral_constant<int, 1>{});
+        if constexpr (Cfg::PC > 2) {
+          piece(std::integral_constant<int, 2>{});
+          piece(std::integral_constant<int, 3>{});
         }
         // the row sum, off the path to P.V
         float2 sum4[4];
