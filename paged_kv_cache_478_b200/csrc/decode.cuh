@@ -388,12 +388,16 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
       if (threadIdx.x == 0) {
         int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
         __threadfence();
-        const int arrived = atomicAdd(cnt, 1) + 1;  // shared-prefix partials are already written
+        const int arrived = atomicAdd(cnt, 1) + 1;  // own partitions only
         s_merge = arrived == ni && !s_abort;
         if (arrived == ni) *cnt = 0;  // re-arm for the next launch on this plan
       }
       __syncthreads();
       if (s_merge && kvh < HK) {
+        // shared-prefix partials come from the preceding launch, which this
+        // one may overlap (programmatic dependent launch): wait for it to
+        // complete before reading them (returns at once otherwise)
+        if (np > ni) grid_dependency_wait();
         __threadfence();
         merge_partitions<T, D>(a, (int64_t)s * HQ + hq, np, lane);
       }

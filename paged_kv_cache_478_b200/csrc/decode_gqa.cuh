@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
       }
       __syncthreads();
       if (s_merge && kvh < HK) {
+        if (np > ni) grid_dependency_wait();  // shared-prefix partials: see the MHA kernel
         __threadfence();
         for (int j = 0; j < G; ++j) merge_partitions<T, D>(a, (int64_t)s * HQ + kvh * G + j, np, lane);
       }

@@ -75,6 +75,20 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the preceding kernel in its stream still
+// runs, once every CTA of that kernel has called grid_dependents_launch() or
+// exited.  grid_dependency_wait() returns when the preceding kernel has
+// completed and its memory operations are visible; without such a launch it
+// returns at once.  The preceding kernel's CTAs are all resident by then and
+// wait on nothing, so the wait ends.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- 16-byte chunks of fp32 / fp16 / bf16 ------------------------------------------
 
 template <typename T>

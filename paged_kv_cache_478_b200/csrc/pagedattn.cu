@@ -196,8 +196,33 @@ cudaError_t set_gqa_attrs() {
                               (int)GqaConfig<T, D, kGqaStages>::smem_bytes(kMaxPartition));
 }
 
+// Launch a persistent decode kernel.  With `overlap`, it is a programmatic
+// dependent launch on the preceding kernel of the stream (the shared-prefix
+// kernel): its CTAs may start while that kernel runs, and wait for it only
+// before merging a sequence that has shared-prefix partials.
+template <typename K>
+cudaError_t launch_decode_grid(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
+                               const DecodeArgs& a, bool overlap) {
+  if (!overlap) {
+    kernel<<<grid, threads, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 template <typename T, int D>
-cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
+cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream,
+                       bool overlap = false) {
   using Cfg = GqaConfig<T, D, kGqaStages>;
   auto kernel = paged_decode_gqa_kernel<T, D, kGqaStages>;
   const size_t smem = Cfg::smem_bytes(a.partition_size);
@@ -207,8 +232,7 @@ cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t
   per_sm = std::max(per_sm, 1);
   const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
-  kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_decode_grid(kernel, grid, Cfg::THREADS, smem, stream, a, overlap);
 }
 
 // Once per device, with that device current: resolve the error word's device
@@ -348,7 +372,8 @@ int resolve_max_context(const pa_pool* pool, int32_t max_blocks_per_seq, int32_t
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream,
+                          bool overlap = false) {
   using Cfg = DecodeKernelCfg<T, D, G>;
   auto kernel = decode_kernel_ptr<T, D, G>();
   const size_t smem = Cfg::smem_bytes(a.partition_size);
@@ -358,17 +383,17 @@ cudaError_t launch_decode(const DecodeArgs& a, const DeviceState& dev, cudaStrea
   per_sm = std::max(per_sm, 1);
   const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
-  kernel<<<grid, Cfg::THREADS, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_decode_grid(kernel, grid, Cfg::THREADS, smem, stream, a, overlap);
 }
 
 template <typename T, int D>
-cudaError_t launch_grouped(int G, const DecodeArgs& a, const DeviceState& dev, cudaStream_t s) {
+cudaError_t launch_grouped(int G, const DecodeArgs& a, const DeviceState& dev, cudaStream_t s,
+                           bool overlap = false) {
   switch (G) {
-    case 1: return launch_decode<T, D, 1>(a, dev, s);
-    case 2: return launch_decode<T, D, 2>(a, dev, s);
-    case 4: return launch_decode<T, D, 4>(a, dev, s);
-    default: return launch_decode<T, D, 8>(a, dev, s);
+    case 1: return launch_decode<T, D, 1>(a, dev, s, overlap);
+    case 2: return launch_decode<T, D, 2>(a, dev, s, overlap);
+    case 4: return launch_decode<T, D, 4>(a, dev, s, overlap);
+    default: return launch_decode<T, D, 8>(a, dev, s, overlap);
   }
 }
 
@@ -547,26 +572,26 @@ pa_status launch_plan(const DecodeArgs& a, cudaStream_t s) {
 }
 
 pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState& dev,
-                     cudaStream_t s) {
+                     cudaStream_t s, bool overlap = false) {
   cudaError_t e;
   if (use_gqa_mma(pool)) {
     switch (pool->dtype * 1000 + pool->head_dim) {
-      case PA_F16 * 1000 + 64: e = launch_gqa<__half, 64>(a, dev, s); break;
-      case PA_F16 * 1000 + 128: e = launch_gqa<__half, 128>(a, dev, s); break;
-      case PA_BF16 * 1000 + 64: e = launch_gqa<__nv_bfloat16, 64>(a, dev, s); break;
-      case PA_BF16 * 1000 + 128: e = launch_gqa<__nv_bfloat16, 128>(a, dev, s); break;
+      case PA_F16 * 1000 + 64: e = launch_gqa<__half, 64>(a, dev, s, overlap); break;
+      case PA_F16 * 1000 + 128: e = launch_gqa<__half, 128>(a, dev, s, overlap); break;
+      case PA_BF16 * 1000 + 64: e = launch_gqa<__nv_bfloat16, 64>(a, dev, s, overlap); break;
+      case PA_BF16 * 1000 + 128: e = launch_gqa<__nv_bfloat16, 128>(a, dev, s, overlap); break;
       default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
     }
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode launch");
   }
   switch (pool->dtype * 1000 + pool->head_dim) {
-    case PA_F32 * 1000 + 64: e = launch_grouped<float, 64>(pool->q_per_kv, a, dev, s); break;
-    case PA_F32 * 1000 + 128: e = launch_grouped<float, 128>(pool->q_per_kv, a, dev, s); break;
-    case PA_F16 * 1000 + 64: e = launch_grouped<__half, 64>(pool->q_per_kv, a, dev, s); break;
-    case PA_F16 * 1000 + 128: e = launch_grouped<__half, 128>(pool->q_per_kv, a, dev, s); break;
-    case PA_BF16 * 1000 + 64: e = launch_grouped<__nv_bfloat16, 64>(pool->q_per_kv, a, dev, s); break;
+    case PA_F32 * 1000 + 64: e = launch_grouped<float, 64>(pool->q_per_kv, a, dev, s, overlap); break;
+    case PA_F32 * 1000 + 128: e = launch_grouped<float, 128>(pool->q_per_kv, a, dev, s, overlap); break;
+    case PA_F16 * 1000 + 64: e = launch_grouped<__half, 64>(pool->q_per_kv, a, dev, s, overlap); break;
+    case PA_F16 * 1000 + 128: e = launch_grouped<__half, 128>(pool->q_per_kv, a, dev, s, overlap); break;
+    case PA_BF16 * 1000 + 64: e = launch_grouped<__nv_bfloat16, 64>(pool->q_per_kv, a, dev, s, overlap); break;
     case PA_BF16 * 1000 + 128:
-      e = launch_grouped<__nv_bfloat16, 128>(pool->q_per_kv, a, dev, s);
+      e = launch_grouped<__nv_bfloat16, 128>(pool->q_per_kv, a, dev, s, overlap);
       break;
     default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
   }
@@ -771,7 +796,9 @@ pa_status pa_decode_attention_shared_prefix(
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "shared prefix launch");
   }
-  return launch_run(pool, a, *dev, s);
+  // the decode launch overlaps the shared-prefix kernel (it needs its
+  // partials only to merge)
+  return launch_run(pool, a, *dev, s, a.group_offsets != nullptr);
 }
 
 pa_status pa_prefill_attention(const pa_pool* pool, const void* q, const void* k_pool,

@@ -56,6 +56,9 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
   constexpr int NT = D / 8;        // 8-column output tiles
   constexpr int CHUNKS = D * 2 / 16;  // 16-byte chunks per token row
   extern __shared__ __align__(128) uint8_t smem[];
+  // the decode launch that follows may start now: it reads this kernel's
+  // partials only after waiting for it to complete
+  grid_dependents_launch();
 
   const int G = a.q_per_kv;
   const int g = blockIdx.x / sp.row_tiles;

@@ -310,6 +310,45 @@ def test_shared_prefix_groups_with_gqa_and_a_bad_member(dtype, group):
     assert_parity(out, ref, f"shared prefix {dtype} G={group}")
 
 
+@pytest.mark.parametrize("group", [1, 4])
+def test_shared_prefix_partials_are_read_after_their_kernel(group):
+    """The decode launch may overlap the shared-prefix kernel before it and
+    reads that kernel's partials only once it has completed.  A long shared
+    prefix (125 blocks) with a few own tokens per sequence makes every merge
+    come early, while the shared-prefix kernel may still run; the workspace is
+    poisoned with NaN before each call, so an early read would show."""
+    rng = np.random.default_rng(70 + group)
+    S, H, D, PB = 64, 8, 128, 125
+    HQ = H * group
+    lens = (PB * BS + rng.integers(1, 17, S)).astype(np.int32)
+    nb = PB + S
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((S, PB + 1), -1, dtype=np.int32)
+    tables[:, :PB] = perm[:PB]
+    tables[:, PB] = perm[PB:]
+    groups = pa.pa_find_shared_prefixes(tables, lens)
+    assert groups["num_groups"] == 1 and groups["blocks"].tolist() == [PB]
+    kh = rng.standard_normal((nb, H, BS, D)).astype(np.float16)
+    vh = rng.standard_normal((nb, H, BS, D)).astype(np.float16)
+    qh = rng.standard_normal((S, HQ, D)).astype(np.float16)
+    scale = 1 / math.sqrt(D)
+    ref = oracle.decode_attention(qh, kh, vh, tables, lens, scale)
+    pool = pa.pa_pool_create(nb, BS, H, D, torch.float16)
+    pa.pa_pool_set_query_heads(pool, HQ)
+    kp, vp, q = dev(kh), dev(vh), dev(qh)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(
+        pool, S, PB + 1, groups["max_shared_blocks"]), dtype=torch.uint8, device="cuda")
+    gd = _groups_to_device(groups)
+    for _ in range(3):
+        ws.fill_(0xFF)  # every fp32 partial reads as NaN until written
+        out = torch.full_like(q, float("nan"))
+        pa.pa_decode_attention_shared_prefix(pool, q, kp, vp, dev(tables), dev(lens), gd, scale,
+                                             out, ws)
+        torch.cuda.synchronize()
+        assert pa.pa_device_errors() == 0
+        assert_parity(out, ref, f"shared prefix read after its kernel, G={group}")
+
+
 def test_shared_prefix_group_larger_than_max_group_size():
     """A group with more members than max_group_size (the launch covers that
     many) is reported, and its members still get the right answer alone."""
