@@ -226,8 +226,8 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
  * log-sum-exp.  Three launches on `stream`: the plan, the shared-prefix
  * kernel, and the decode kernel as a programmatic dependent launch that may
  * run alongside the shared-prefix kernel and waits for it before any merge
- * that reads its partials (stream capture keeps that edge).  fp16/bf16 pools
- * only (PA_ERR_UNSUPPORTED for fp32).
+ * that reads its partials.  fp16/bf16 pools only (PA_ERR_UNSUPPORTED for
+ * fp32).
  * max_group_size and max_shared_blocks bound the group sizes and
  * group_blocks (launch sizing); a group beyond either bound is reported
  * (PA_DEVERR_CONTEXT_LEN) and its members attend alone.  A member that is
