@@ -103,3 +103,37 @@ def test_status_strings():
     lib = pa.lib()
     assert lib.pa_status_string(0) == b"PA_OK"
     assert lib.pa_status_string(5) == b"PA_ERR_NO_FREE_BLOCKS"
+
+
+def test_prefill_and_shared_prefix_validate_on_the_host():
+    """Both calls reject bad arguments before their first CUDA call."""
+    lib = pa.lib()
+    f = ctypes.c_float
+    ok = ctypes.c_void_p(0x2000)  # aligned, never dereferenced on these paths
+    p32 = pa.pa_pool_create(16, 16, 2, 64, pa.PA_F32)
+    p16 = pa.pa_pool_create(16, 16, 2, 64, pa.PA_F16)
+
+    def prefill(pool, q=ok, qs=ok, num_seqs=1, num_tokens=8, max_new=8, scale=0.1, out=ok):
+        return lib.pa_prefill_attention(ctypes.byref(pool), q, ok, ok, ok, 4, ok, qs, num_seqs,
+                                        num_tokens, max_new, 0, f(scale), out, None)
+
+    assert prefill(p32) == 2                      # tensor cores: fp16 / bf16 pools only
+    assert prefill(p16, q=None) == 1
+    assert prefill(p16, qs=None) == 1
+    assert prefill(p16, out=None) == 1
+    assert prefill(p16, num_seqs=-1) == 1
+    assert prefill(p16, scale=float("nan")) == 1
+    assert prefill(p16, q=ctypes.c_void_p(0x2008)) == 1  # misaligned
+    assert prefill(p16, q=None, qs=None, out=None, num_tokens=0) == 0  # nothing to do
+
+    def shared(pool, offsets=ok, members=ok, blocks=ok, num_groups=1, ctx=ok):
+        return lib.pa_decode_attention_shared_prefix(
+            ctypes.byref(pool), ok, ok, ok, ok, 4, ctx, 2, offsets, members, 2, blocks, num_groups,
+            2, 2, 0, f(0.1), ok, ok, 1 << 20, 0, None)
+
+    assert shared(p32) == 2                       # the shared blocks go through mma.sync
+    assert shared(p16, offsets=None) == 1
+    assert shared(p16, members=None) == 1
+    assert shared(p16, blocks=None) == 1
+    assert shared(p16, ctx=None) == 1
+    assert shared(p16, num_groups=-1) == 1
