@@ -166,7 +166,10 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
  * A plan stays valid for any number of planned calls with the same pool
  * geometry (heads, head_dim, dtype), num_seqs, max_blocks_per_seq,
  * max_context_len and partition_size, issued in stream order on the same
- * workspace; each planned call leaves the plan ready for the next.
+ * workspace; each planned call leaves the plan ready for the next.  The
+ * library records the parameters of every plan it writes, per workspace: a
+ * planned call whose arguments resolve to others, or that finds no plan in
+ * its workspace, returns PA_ERR_INVALID_ARG without launching.
  */
 pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32_t num_seqs,
                          int32_t max_blocks_per_seq, int32_t max_context_len,

@@ -9,7 +9,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "cache_ops.cuh"
 #include "decode.cuh"
@@ -565,10 +567,59 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
   return PA_OK;
 }
 
-pa_status launch_plan(const DecodeArgs& a, cudaStream_t s) {
+// ---- plans recorded per workspace ------------------------------------------------
+// The work items, partial slots and merge counters a planned call reads were
+// laid out by the plan in its workspace.  Every plan the library writes is
+// recorded under the workspace's plan address with the parameters it was made
+// with, and a planned call that resolves to other parameters, or finds no
+// plan there, is refused rather than run on a layout it does not match.
+struct PlanKey {
+  int32_t num_seqs, max_blocks_per_seq, max_context_len, partition_size, max_parts, head_groups,
+      heads, q_per_kv, head_dim, dtype, device;
+};
+
+PlanKey plan_key(const pa_pool* pool, const DecodeArgs& a) {
+  int dev = -1;
+  cudaGetDevice(&dev);
+  return PlanKey{a.num_seqs,   a.max_blocks_per_seq, a.max_context_len, a.partition_size,
+                 a.max_parts,  a.head_groups,        pool->heads,       pool->q_per_kv,
+                 pool->head_dim, (int32_t)pool->dtype, dev};
+}
+
+std::mutex g_plan_mutex;
+std::unordered_map<const void*, PlanKey>& plan_registry() {
+  static std::unordered_map<const void*, PlanKey> plans;
+  return plans;
+}
+
+pa_status check_plan(const pa_pool* pool, const DecodeArgs& a, const char* who) {
+  const PlanKey want = plan_key(pool, a);
+  std::lock_guard<std::mutex> lock(g_plan_mutex);
+  const auto it = plan_registry().find(a.plan);
+  char buf[200];
+  if (it == plan_registry().end()) {
+    std::snprintf(buf, sizeof buf, "%s: no plan was written to this workspace (pa_decode_plan)",
+                  who);
+    return fail(PA_ERR_INVALID_ARG, buf);
+  }
+  if (std::memcmp(&it->second, &want, sizeof want) != 0) {
+    std::snprintf(buf, sizeof buf,
+                  "%s: the arguments differ from the plan's in this workspace (sequences, "
+                  "table width, max_context_len, partition_size and pool must match)",
+                  who);
+    return fail(PA_ERR_INVALID_ARG, buf);
+  }
+  return PA_OK;
+}
+
+pa_status launch_plan(const pa_pool* pool, const DecodeArgs& a, cudaStream_t s) {
   decode_plan_kernel<<<1, 1024, (a.partition_size / kBlock + 1) * sizeof(int32_t), s>>>(a);
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode plan launch");
+  if (e != cudaSuccess) return cuda_fail(e, "decode plan launch");
+  const PlanKey k = plan_key(pool, a);
+  std::lock_guard<std::mutex> lock(g_plan_mutex);
+  plan_registry()[a.plan] = k;
+  return PA_OK;
 }
 
 pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState& dev,
@@ -635,7 +686,7 @@ pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32
                                 partition_size, workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
   a.context_lens = context_lens;
-  return launch_plan(a, static_cast<cudaStream_t>(stream));
+  return launch_plan(pool, a, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const void* k_pool,
@@ -653,6 +704,7 @@ pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const 
   st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
                       workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
+  if ((st = check_plan(pool, a, "pa_decode_attention_planned")) != PA_OK) return st;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   return launch_run(pool, a, *dev, static_cast<cudaStream_t>(stream));
 }
@@ -677,7 +729,7 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
   a.context_lens = context_lens;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = launch_plan(a, s)) != PA_OK) return st;
+  if ((st = launch_plan(pool, a, s)) != PA_OK) return st;
   return launch_run(pool, a, *dev, s);
 }
 
@@ -701,6 +753,7 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
   st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
                       workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
+  if ((st = check_plan(pool, a, "pa_decode_append_attention_planned")) != PA_OK) return st;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   a.k_new = k_new;
   a.v_new = v_new;
@@ -764,7 +817,7 @@ pa_status pa_decode_attention_shared_prefix(
   }
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = launch_plan(a, s)) != PA_OK) return st;
+  if ((st = launch_plan(pool, a, s)) != PA_OK) return st;
   if (a.group_offsets != nullptr) {
     SharedPrefixArgs sp;
     sp.group_offsets = group_offsets;

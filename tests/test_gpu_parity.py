@@ -277,6 +277,31 @@ def test_wait_limit_reports_a_timeout_and_the_context_survives():
     assert_parity(out, ref, "after timeout")
 
 
+def test_planned_call_refuses_arguments_that_differ_from_the_plan():
+    """A planned call reads the work items, partial slots and merge counters the
+    plan laid out; with other partition or length bounds it is refused on the
+    host instead of running on a layout it does not match."""
+    case = syn.decode_case(5, [40, 300, 17, 129], heads=2, head_dim=64, dtype=np.float16)
+    NB, H, BS, D = case["k_pool"].shape
+    pool = pa.pa_pool_create(NB, BS, H, D, torch.float16)
+    bt, cl = dev(case["block_tables"]), dev(case["context_lens"])
+    kp, vp, q = dev(case["k_pool"]), dev(case["v_pool"]), dev(case["q"])
+    ws = workspace_for(pool, 4, bt.shape[1], partition_size=32)  # large enough for both
+    out = torch.empty_like(q)
+    pa.pa_decode_plan(pool, cl, bt.shape[1], ws, partition_size=128)
+    with pytest.raises(pa.PagedAttnError, match="differ"):
+        pa.pa_decode_attention_planned(pool, q, kp, vp, bt, case["scale"], out, ws,
+                                       partition_size=32)
+    with pytest.raises(pa.PagedAttnError, match="differ"):
+        pa.pa_decode_attention_planned(pool, q, kp, vp, bt, case["scale"], out, ws,
+                                       max_context_len=160, partition_size=128)
+    pa.pa_decode_attention_planned(pool, q, kp, vp, bt, case["scale"], out, ws, partition_size=128)
+    assert pa.pa_device_errors() == 0
+    ref = oracle.decode_attention(case["q"], case["k_pool"], case["v_pool"], case["block_tables"],
+                                  case["context_lens"], case["scale"])
+    assert_parity(out, ref, "planned call matching its plan")
+
+
 def test_plan_once_run_many_layers_matches_single_calls():
     """One plan serves several layers that share lengths and tables."""
     case = syn.single_layer_case(seed=4, num_seqs=24)
