@@ -7,14 +7,17 @@
 // contractions, S = Q.K^T and O = P.V.
 //
 // A work item = (sequence, query head, 256 new queries as two 128-row tiles).
-// One persistent CTA per SM walks the items heaviest first, with specialised
-// warps:
+// CTAs walk the items heaviest first (fp16: one persistent CTA per SM; bf16:
+// the grid covers every item, so each CTA's walk is one item), with
+// specialised warps:
 //   * warps 0-3 and 4-7: two softmax warpgroups, one per query tile; thread r
 //     of a group owns query row r (TMEM lane r).  Each reads its row of S
 //     (128 keys) from TMEM, applies the causal mask and the online softmax in
 //     fp32 (log2 domain) and writes its row of P (fp16/bf16 pairs) back over
-//     S in TMEM, where the P.V product takes its A operand from; at the end
-//     of an item it writes its rows of O out and frees O for the next item;
+//     S in TMEM, where the P.V product takes its A operand from.  P is handed
+//     over in two 64-key pieces, each on its own mbarrier, so that P.V of the
+//     first runs while the second is computed.  At the end of an item the
+//     group writes its rows of O out and frees O for the next item;
 //   * warp 8: the loader.  It loads each item's Q tiles and streams the paged
 //     K and V rows of each 128-key tile with TMA tensor copies (one 16-row box
 //     per physical block and 64-wide slice of head_dim, hardware 128-byte
