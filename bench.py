@@ -41,8 +41,11 @@ S, LAYERS, H, D, BS = 200, 32, 32, 128, 16
 ELT = 2  # fp16
 WORKLOAD = "full 32-layer decode step: 200 requests, 32 layers x 32 heads x 128 fp16, block 16"
 METRIC = "paged-decode KV-read GB/s (% of B200 HBM peak); decode tokens/s"
-DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_478_b200", "csrc", "decode.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "paged_decode_kernel_full_step.md")
+CSRC = os.path.join(ROOT, "paged_kv_cache_478_b200", "csrc")
+# the decode kernel's device code: its traffic figure holds while these are unchanged
+DECODE_SOURCES = ("decode.cuh", "plan.cuh", "device_utils.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+CLOCK_PERIOD_MS = 50
 
 
 def parse():
@@ -82,27 +85,28 @@ def algorithmic_bytes_per_launch(lens):
 
 
 def decode_source_hash():
-    with open(DECODE_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256[:16] over the decode kernel's device sources, in a fixed order."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def committed_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
+    """DRAM bytes per decode launch from the committed ncu figure
+    (profiles/decode_traffic.json), if it was taken on the current kernel
+    sources; else None."""
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    vals = {}
-    for line in text.splitlines():
-        if ": " in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(": ", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("decode.cuh sha256[:16]") != decode_source_hash():
+    if rec.get("sources_sha256_16") != decode_source_hash():
         return None
     try:
-        return float(vals["dram bytes per launch (read + write)"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -121,8 +125,9 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(CLOCK_PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t0 = time.perf_counter()
         except OSError:
             self.proc = None
 
@@ -150,7 +155,9 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
         loaded = [r for r in rows if r[2] > 200.0] or rows
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "period_ms": CLOCK_PERIOD_MS,
+                "window_s": round(time.perf_counter() - self.t0, 3),
                 "power_w_max": max(r[2] for r in rows)}
 
 
@@ -172,13 +179,15 @@ def time_oracle(case, reps=1, threads=None):
     kp, vp = case["k_pool"].copy(), case["v_pool"].copy()
     slots = np.array([oracle.slot_of_c(case["block_tables"][s], int(L) - 1)
                       for s, L in enumerate(case["context_lens"])], dtype=np.int32)
-    t0 = time.perf_counter()
+    t0, c0 = time.perf_counter(), time.process_time()
     for _ in range(reps):
         oracle.reshape_and_cache(case["k_new"], case["v_new"], slots, kp, vp)
         oracle.decode_attention(case["q"], kp, vp, case["block_tables"], case["context_lens"],
                                 case["scale"], num_threads=cores)
-    dt = (time.perf_counter() - t0) / reps
-    return kv_bytes(case["context_lens"]) / dt / 1e9, cores
+    wall = time.perf_counter() - t0
+    # effective parallelism: CPU time of all the process's threads over wall time
+    eff = (time.process_time() - c0) / wall if wall > 0 else 0.0
+    return kv_bytes(case["context_lens"]) / (wall / reps) / 1e9, cores, eff
 
 
 def run_reference(args):
@@ -192,13 +201,12 @@ def run_reference(args):
     case = oracle_sample_case(0, n_sample)
     for _ in range(args.warmup):
         time_oracle(case)
-    t0 = time.perf_counter()
-    vals = []
+    t0, c0 = time.perf_counter(), time.process_time()
     cores = 1
     for _ in range(args.steps):
-        v, cores = time_oracle(case)
-        vals.append(v)
+        _, cores, _ = time_oracle(case)
     elapsed = time.perf_counter() - t0
+    eff = (time.process_time() - c0) / elapsed if elapsed > 0 else 0.0
     value = kv_bytes(case["context_lens"]) * args.steps / elapsed / 1e9
     sample = (f"one layer of the first {n_sample} of the 200 requests "
               f"({int(case['context_lens'].sum())} cached tokens, 32 heads x 128 fp16) per step")
@@ -209,7 +217,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "sample": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "effective_cores": round(eff, 2), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -326,6 +334,7 @@ def run_ours(args):
         step()
     assert pa.pa_device_errors() == 0, "device error bits set during warm-up"
 
+    # clocks are sampled across the three timed legs (eager, graph, e2e)
     uuid = torch.cuda.get_device_properties(dev).uuid
     sampler = ClockSampler(f"GPU-{uuid}" if not str(uuid).startswith("GPU-") else str(uuid))
     sampler.start()
@@ -341,7 +350,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     errs = pa.pa_device_errors()
     assert errs == 0, f"device error bits {errs:#x}"
@@ -359,17 +367,23 @@ def run_ours(args):
     graph = run_graph(args, torch, step, stream, lens, n_layers, world, dev)
     e2e = None if args.no_e2e else run_e2e(args, pa, torch, pool, kpools, vpools, tables, lens,
                                           ws, ps, world, dev)
+    clocks = sampler.stop()
+    if clocks is not None:
+        clocks["legs"] = "eager" + (", graph" if graph and "error" not in graph else "") + \
+                         ("" if args.no_e2e else ", e2e")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         case = oracle_sample_case(0, 40)
-        v, cores = time_oracle(case)
+        v, cores, eff = time_oracle(case)
         one = oracle_sample_case(0, 4)
-        v1, _ = time_oracle(one, threads=1)
-        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+        v1, _, eff1 = time_oracle(one, threads=1)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+               "effective_cores": round(eff, 2), "kind": "oracle",
                "sample": f"one layer of the first 40 of the 200 requests "
                          f"({int(case['context_lens'].sum())} cached tokens), fp64 C oracle, "
                          f"OpenMP over (sequence, head)",
                "single_thread": {"value": round(v1, 4), "unit": "GB/s", "cores": 1,
+                                 "effective_cores": round(eff1, 2),
                                  "sample": f"one layer of the first 4 requests "
                                            f"({int(one['context_lens'].sum())} cached tokens)"}}
 

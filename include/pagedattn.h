@@ -69,6 +69,9 @@ typedef enum {
 #define PA_DEVERR_CONTEXT_LEN 0x4u /* context_len < 0 or above the table / max bound */
 #define PA_DEVERR_PAIR 0x8u        /* copy_blocks pair outside the pool */
 #define PA_DEVERR_TIMEOUT 0x10u    /* an mbarrier wait ran past its limit */
+#define PA_DEVERR_PLAN 0x20u       /* the workspace holds no plan this launch may run, or a
+                                      damaged entry of one (the launch skips what it cannot
+                                      trust) */
 
 /* Plain value descriptor of one K or V pool (the two share it). */
 typedef struct pa_pool {
@@ -170,6 +173,17 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
  * library records the parameters of every plan it writes, per workspace: a
  * planned call whose arguments resolve to others, or that finds no plan in
  * its workspace, returns PA_ERR_INVALID_ARG without launching.
+ * Each plan also carries a stamp, a number the host draws for it, in the
+ * workspace header.  The kernels check it on the device: a launch that
+ * finds another stamp (the workspace was freed and reused, overwritten or
+ * zeroed since the plan was written, or holds an older plan) raises
+ * PA_DEVERR_PLAN and touches neither the workspace nor out.  Every plan
+ * entry a launch uses is bounds-checked before it indexes anything; a
+ * damaged entry raises PA_DEVERR_PLAN and its work item is skipped.
+ * After PA_DEVERR_TIMEOUT the outputs of that launch are undefined, and the
+ * plan is marked so that later planned launches on it are refused
+ * (PA_DEVERR_PLAN) until pa_decode_plan rewrites it: a launch that gave up
+ * may leave the split-K merge counters mid-count.
  */
 pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32_t num_seqs,
                          int32_t max_blocks_per_seq, int32_t max_context_len,

@@ -29,6 +29,7 @@ PA_DEVERR_SLOT = 0x2
 PA_DEVERR_CONTEXT_LEN = 0x4
 PA_DEVERR_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
+PA_DEVERR_PLAN = 0x20
 
 
 class PagedAttnError(RuntimeError):

@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   __shared__ int32_t s_item;
   __shared__ int32_t s_abort;
   __shared__ int32_t s_merge;
+  __shared__ int32_t s_plan_ok;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -186,15 +187,20 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   const int HQ = a.heads * G;           // query heads
   const int PS = a.partition_size;
 
+  int32_t next = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < RINGS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
     s_abort = 0;
+    // a plan that is not this launch's, or that an earlier launch gave up
+    // on, is not run: nothing in the workspace is touched
+    s_plan_ok = plan_header_ok(a);
+    if (s_plan_ok) next = atomicAdd(&a.plan->work_counter, 1);
+    else atomicOr(a.err, PA_DEVERR_PLAN);
   }
-  int32_t next = 0;
-  if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
-  const int32_t num_items = a.plan->num_items;
   __syncthreads();
+  if (!s_plan_ok) return;
+  const int32_t num_items = a.plan->num_items;
 
   uint32_t fills = 0;  // stage fills this ring has consumed so far (drives ring slot + parity)
   uint8_t* my_stages = stages + ring * NSTAGE * Cfg::STAGE_BYTES;
@@ -209,19 +215,21 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
     const int item = s_item;
     if (item >= num_items || s_abort) break;
 
-    const int2 pr = a.pairs[item / a.head_groups];
+    PlanItem it;
+    if (!plan_item(a, item, &it)) {  // a damaged plan entry: report and skip the item
+      if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_PLAN);
+      __syncthreads();
+      continue;
+    }
     const int g = item % a.head_groups;
-    const int s = pr.x, p = pr.y;
-    const int L = a.lens[s];
-    const int np = a.nparts[s];
-    const int ni = a.nitems[s];
+    const int s = it.s, p = it.p, L = it.L, np = it.np, ni = it.ni;
     const bool split = np > 1;
-    const int tok0 = a.base[s] + p * PS;
+    const int tok0 = it.base + p * PS;
     const int ntok = max(0, min(L, tok0 + PS) - tok0);
     const int nblk = (ntok + kBlock - 1) / kBlock;
     const int blk0 = tok0 / kBlock;
     // the item holding the sequence's last token appends the new one (fused mode)
-    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1;
+    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1 && tok0 + ntok == L;
     const int new_row = (L - 1) % kBlock;  // in-block offset of the appended token
 
     // block-table slice of this partition, bounds-checked once
@@ -345,10 +353,14 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         }
       }
       if (!ok) {
-        // give up on this item: report, let the copies already issued land, stop the CTA
+        // give up on this item: report, let the copies already issued land,
+        // stop the CTA, and mark the plan so that no merge trusts its
+        // counters again until it is rewritten
         if (lane == 0) {
           atomicOr(a.err, PA_DEVERR_TIMEOUT);
           s_abort = 1;
+          a.plan->poisoned = 1;
+          __threadfence();
         }
         const int issued = min(nblk, i + NSTAGE);
         for (int j = i; j < issued; ++j) {
@@ -389,7 +401,9 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
         __threadfence();
         const int arrived = atomicAdd(cnt, 1) + 1;  // own partitions only
-        s_merge = arrived == ni && !s_abort;
+        __threadfence();
+        // no merge once any CTA of this launch gave up (its partial may be missing)
+        s_merge = arrived == ni && !s_abort && *(volatile int32_t*)&a.plan->poisoned == 0;
         if (arrived == ni) *cnt = 0;  // re-arm for the next launch on this plan
       }
       __syncthreads();

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
   __shared__ int32_t s_item;
   __shared__ int32_t s_abort;
   __shared__ int32_t s_merge;
+  __shared__ int32_t s_plan_ok;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -70,15 +71,18 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
   const int HK = a.heads, HQ = a.heads * G;
   const int PS = a.partition_size;
 
+  int32_t next = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
     s_abort = 0;
+    s_plan_ok = plan_header_ok(a);  // see the MHA kernel
+    if (s_plan_ok) next = atomicAdd(&a.plan->work_counter, 1);
+    else atomicOr(a.err, PA_DEVERR_PLAN);
   }
-  int32_t next = 0;
-  if (threadIdx.x == 0) next = atomicAdd(&a.plan->work_counter, 1);
-  const int32_t num_items = a.plan->num_items;
   __syncthreads();
+  if (!s_plan_ok) return;
+  const int32_t num_items = a.plan->num_items;
 
   uint32_t fills = 0;
   uint8_t* my_stages = stages + warp * NSTAGE * Cfg::STAGE_BYTES;
@@ -96,18 +100,20 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
     const int item = s_item;
     if (item >= num_items || s_abort) break;
 
-    const int2 pr = a.pairs[item / a.head_groups];
+    PlanItem it;
+    if (!plan_item(a, item, &it)) {  // a damaged plan entry: report and skip the item
+      if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_PLAN);
+      __syncthreads();
+      continue;
+    }
     const int g = item % a.head_groups;
-    const int s = pr.x, p = pr.y;
-    const int L = a.lens[s];
-    const int np = a.nparts[s];
-    const int ni = a.nitems[s];
+    const int s = it.s, p = it.p, L = it.L, np = it.np, ni = it.ni;
     const bool split = np > 1;
-    const int tok0 = a.base[s] + p * PS;
+    const int tok0 = it.base + p * PS;
     const int ntok = max(0, min(L, tok0 + PS) - tok0);
     const int nblk = (ntok + kBlock - 1) / kBlock;
     const int blk0 = tok0 / kBlock;
-    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1;
+    const bool append = a.k_new != nullptr && L > 0 && p == ni - 1 && tok0 + ntok == L;
     const int new_row = (L - 1) % kBlock;
 
     for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
@@ -275,9 +281,11 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
         if (i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
       }
       if (!ok) {
-        if (lane == 0) {
+        if (lane == 0) {  // as in the MHA kernel: report, stop, and poison the plan
           atomicOr(a.err, PA_DEVERR_TIMEOUT);
           s_abort = 1;
+          a.plan->poisoned = 1;
+          __threadfence();
         }
         const int issued = min(nblk, i + NSTAGE);
         for (int j = i; j < issued; ++j) {
@@ -312,7 +320,8 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
         int32_t* cnt = a.merge_cnt + (int64_t)s * a.head_groups + g;
         __threadfence();
         const int arrived = atomicAdd(cnt, 1) + 1;
-        s_merge = arrived == ni && !s_abort;
+        __threadfence();
+        s_merge = arrived == ni && !s_abort && *(volatile int32_t*)&a.plan->poisoned == 0;
         if (arrived == ni) *cnt = 0;
       }
       __syncthreads();

@@ -6,11 +6,13 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <unordered_map>
 
 #include "cache_ops.cuh"
@@ -586,39 +588,63 @@ PlanKey plan_key(const pa_pool* pool, const DecodeArgs& a) {
                  pool->head_dim, (int32_t)pool->dtype, dev};
 }
 
+struct PlanRecord {
+  PlanKey key;
+  uint64_t stamp;  // written into the plan's header; the kernels run only on a matching one
+};
+
 std::mutex g_plan_mutex;
-std::unordered_map<const void*, PlanKey>& plan_registry() {
-  static std::unordered_map<const void*, PlanKey> plans;
+std::unordered_map<const void*, PlanRecord>& plan_registry() {
+  static std::unordered_map<const void*, PlanRecord> plans;
   return plans;
 }
 
-pa_status check_plan(const pa_pool* pool, const DecodeArgs& a, const char* who) {
-  const PlanKey want = plan_key(pool, a);
+// A fresh number for every plan: a random per-process high half (so a stale
+// plan left in reused memory by another process does not match) and a
+// counter that never yields zero (so a zeroed workspace does not match).
+uint64_t next_plan_stamp() {
+  static const uint64_t salt = [] {
+    std::random_device rd;
+    return (uint64_t)rd() << 32;
+  }();
+  static std::atomic<uint32_t> counter{0};
+  uint32_t n = ++counter;
+  if (n == 0) n = ++counter;
+  return salt | n;
+}
+
+// On success a->stamp is the stamp of the plan recorded for a's workspace.
+pa_status check_plan(const pa_pool* pool, DecodeArgs* a, const char* who) {
+  const PlanKey want = plan_key(pool, *a);
   std::lock_guard<std::mutex> lock(g_plan_mutex);
-  const auto it = plan_registry().find(a.plan);
+  const auto it = plan_registry().find(a->plan);
   char buf[200];
   if (it == plan_registry().end()) {
     std::snprintf(buf, sizeof buf, "%s: no plan was written to this workspace (pa_decode_plan)",
                   who);
     return fail(PA_ERR_INVALID_ARG, buf);
   }
-  if (std::memcmp(&it->second, &want, sizeof want) != 0) {
+  if (std::memcmp(&it->second.key, &want, sizeof want) != 0) {
     std::snprintf(buf, sizeof buf,
                   "%s: the arguments differ from the plan's in this workspace (sequences, "
                   "table width, max_context_len, partition_size and pool must match)",
                   who);
     return fail(PA_ERR_INVALID_ARG, buf);
   }
+  a->stamp = it->second.stamp;
   return PA_OK;
 }
 
-pa_status launch_plan(const pa_pool* pool, const DecodeArgs& a, cudaStream_t s) {
-  decode_plan_kernel<<<1, 1024, (a.partition_size / kBlock + 1) * sizeof(int32_t), s>>>(a);
+// Write a plan under a fresh stamp (left in a->stamp for the launches that
+// follow in the same call) and record it for the workspace.
+pa_status launch_plan(const pa_pool* pool, DecodeArgs* a, cudaStream_t s) {
+  a->stamp = next_plan_stamp();
+  decode_plan_kernel<<<1, 1024, (a->partition_size / kBlock + 1) * sizeof(int32_t), s>>>(*a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode plan launch");
-  const PlanKey k = plan_key(pool, a);
+  const PlanKey k = plan_key(pool, *a);
   std::lock_guard<std::mutex> lock(g_plan_mutex);
-  plan_registry()[a.plan] = k;
+  plan_registry()[a->plan] = PlanRecord{k, a->stamp};
   return PA_OK;
 }
 
@@ -686,7 +712,7 @@ pa_status pa_decode_plan(const pa_pool* pool, const int32_t* context_lens, int32
                                 partition_size, workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
   a.context_lens = context_lens;
-  return launch_plan(pool, a, static_cast<cudaStream_t>(stream));
+  return launch_plan(pool, &a, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const void* k_pool,
@@ -704,7 +730,7 @@ pa_status pa_decode_attention_planned(const pa_pool* pool, const void* q, const 
   st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
                       workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
-  if ((st = check_plan(pool, a, "pa_decode_attention_planned")) != PA_OK) return st;
+  if ((st = check_plan(pool, &a, "pa_decode_attention_planned")) != PA_OK) return st;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   return launch_run(pool, a, *dev, static_cast<cudaStream_t>(stream));
 }
@@ -729,7 +755,7 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
   a.context_lens = context_lens;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = launch_plan(pool, a, s)) != PA_OK) return st;
+  if ((st = launch_plan(pool, &a, s)) != PA_OK) return st;
   return launch_run(pool, a, *dev, s);
 }
 
@@ -753,7 +779,7 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
   st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
                       workspace, workspace_bytes, &a, &dev);
   if (st != PA_OK) return st;
-  if ((st = check_plan(pool, a, "pa_decode_append_attention_planned")) != PA_OK) return st;
+  if ((st = check_plan(pool, &a, "pa_decode_append_attention_planned")) != PA_OK) return st;
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   a.k_new = k_new;
   a.v_new = v_new;
@@ -817,7 +843,7 @@ pa_status pa_decode_attention_shared_prefix(
   }
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = launch_plan(pool, a, s)) != PA_OK) return st;
+  if ((st = launch_plan(pool, &a, s)) != PA_OK) return st;
   if (a.group_offsets != nullptr) {
     SharedPrefixArgs sp;
     sp.group_offsets = group_offsets;
@@ -998,6 +1024,7 @@ pa_status pa_decode_attention_static(const pa_pool* pool, const void* q, const v
                                      void* out, int32_t partition_size, void* stream) {
   CallRange range("pa_decode_attention_static");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "pa_decode_attention_static: num_seqs < 0");
+  if (num_seqs == 0) return check_pool(pool);  // as pa_decode_attention: nothing to launch
   size_t need = 0;
   pa_status st = pa_decode_workspace_bytes(pool, num_seqs, max_blocks_per_seq, max_context_len,
                                            partition_size, &need);
@@ -1032,6 +1059,9 @@ pa_status pa_device_errors(void* stream, uint32_t* flags) {
   if (e != cudaSuccess) return cuda_fail(e, "pa_device_errors");
   *flags = v;
   if (v & PA_DEVERR_TIMEOUT) return fail(PA_ERR_TIMEOUT, "a device-side wait timed out");
+  if (v & PA_DEVERR_PLAN)
+    return fail(PA_ERR_OUT_OF_BOUNDS,
+                "a planned launch found no valid plan in its workspace, or a damaged entry");
   if (v) return fail(PA_ERR_OUT_OF_BOUNDS, "a device-side bounds check fired");
   return PA_OK;
 }

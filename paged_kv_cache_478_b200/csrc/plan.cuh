@@ -23,6 +23,9 @@ struct PlanHeader {
   int32_t num_items;     // num_pairs * head_groups
   int32_t work_counter;  // next item index to hand out
   int32_t done_counter;  // CTAs that have left the work loop
+  uint64_t stamp;        // the host's number for this plan; a launch runs only on its own plan
+  int32_t poisoned;      // a launch on this plan gave up on a wait: refused until re-planned
+  int32_t reserved;
 };
 
 struct DecodeArgs {
@@ -64,7 +67,43 @@ struct DecodeArgs {
   int32_t max_parts;
   int32_t max_context_len;
   float scale_log2;  // scale * log2(e)
+  uint64_t stamp;    // number of the plan the host expects in the workspace
 };
+
+// Checks a CTA makes before it trusts the plan in the workspace: the header
+// carries the stamp this launch was given, no earlier launch on the plan gave
+// up, and the item count is within what the workspace can hold.  Any failure
+// raises PA_DEVERR_PLAN and the launch touches nothing in the workspace.
+__device__ __forceinline__ bool plan_header_ok(const DecodeArgs& a) {
+  const PlanHeader* h = a.plan;
+  const int64_t cap = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
+  return h->stamp == a.stamp && h->poisoned == 0 && h->num_items >= 0 && h->num_items <= cap;
+}
+
+// One work item's view of the plan, bounds-checked so that a damaged
+// workspace can cost the result but never an access outside the caller's
+// buffers: the sequence is in range, its clamped length within the table
+// and max_context_len, its own part starts on a block boundary inside the
+// context, and the partition index and partial counts fit the workspace.
+struct PlanItem {
+  int s, p, L, np, ni, base;
+};
+
+__device__ __forceinline__ bool plan_item(const DecodeArgs& a, int item, PlanItem* it) {
+  const int2 pr = a.pairs[item / a.head_groups];
+  it->s = pr.x;
+  it->p = pr.y;
+  if (pr.x < 0 || pr.x >= a.num_seqs) return false;
+  it->L = a.lens[pr.x];
+  it->np = a.nparts[pr.x];
+  it->ni = a.nitems[pr.x];
+  it->base = a.base[pr.x];
+  const int64_t cap = min((int64_t)a.max_context_len, (int64_t)a.max_blocks_per_seq * kBlock);
+  return it->L >= 0 && it->L <= cap && it->base >= 0 && it->base <= it->L &&
+         it->base % kBlock == 0 && it->ni >= 1 && it->np >= it->ni && it->np <= a.max_parts &&
+         pr.y >= 0 && pr.y < it->ni &&
+         (int64_t)it->base + (int64_t)pr.y * a.partition_size <= it->L;
+}
 
 // ---- plan: one CTA orders the work ------------------------------------------------
 
@@ -75,7 +114,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
   const int nb = PS / kBlock;
   for (int i = threadIdx.x; i <= nb; i += blockDim.x) bucket[i] = 0;
   if (threadIdx.x == 0) n_full = 0;
-  const int cap = min(a.max_context_len, a.max_blocks_per_seq * kBlock);
+  const int cap = (int)min((int64_t)a.max_context_len, (int64_t)a.max_blocks_per_seq * kBlock);
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     int L = a.context_lens[s];
     if (L < 0 || L > cap) {
@@ -159,6 +198,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
     a.plan->num_items = run * a.head_groups;
     a.plan->work_counter = 0;
     a.plan->done_counter = 0;
+    a.plan->stamp = a.stamp;
+    a.plan->poisoned = 0;
   }
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {

@@ -59,6 +59,10 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
   // the decode launch that follows may start now: it reads this kernel's
   // partials only after waiting for it to complete
   grid_dependents_launch();
+  if (!plan_header_ok(a)) {  // not the plan this call wrote: touch nothing
+    if (threadIdx.x == 0) atomicOr(a.err, PA_DEVERR_PLAN);
+    return;
+  }
 
   const int G = a.q_per_kv;
   const int g = blockIdx.x / sp.row_tiles;
@@ -224,6 +228,10 @@ __global__ void __launch_bounds__(128) shared_prefix_kernel(SharedPrefixArgs sp,
     const int s = row_s[h2];
     const int64_t sh = (int64_t)s * HQ + row_hq[h2];
     const int slot = a.nitems[s] + chunk;
+    if (a.nitems[s] < 1 || slot >= a.max_parts) {  // a damaged plan entry
+      atomicOr(a.err, PA_DEVERR_PLAN);
+      continue;
+    }
     float* dst = a.part_acc + (sh * a.max_parts + slot) * D + (lane & 3) * 2;
 #pragma unroll
     for (int j = 0; j < NT; ++j)

@@ -3,15 +3,18 @@
     python -m paged_kv_cache_478_b200.kernel_bench prefill [--small]
     python -m paged_kv_cache_478_b200.kernel_bench gqa
     python -m paged_kv_cache_478_b200.kernel_bench shared-prefix
-    python -m paged_kv_cache_478_b200.kernel_bench long-context
-    python -m paged_kv_cache_478_b200.kernel_bench single-layer
-    python -m paged_kv_cache_478_b200.kernel_bench cache-ops
+    python -m paged_kv_cache_478_b200.kernel_bench long-context [--profile]
+    python -m paged_kv_cache_478_b200.kernel_bench single-layer [--profile]
+    python -m paged_kv_cache_478_b200.kernel_bench cache-ops [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench decode-dtypes
 
 Each line printed is one JSON object.  These are the measurements behind the
 per-kernel tables of the design notes; the headline decode step is bench.py.
 `prefill --small` runs three launches of one small case (2 prompts x 2048
 tokens) and prints nothing timed: it is the command the profiler captures.
+`--profile` does the same for the other workloads: the same inputs, a few
+plain launches (no CUDA graph, no timing), so that a profiler capture of
+one launch stays small and ends by itself.
 """
 from __future__ import annotations
 
@@ -203,7 +206,16 @@ def shared_prefix():
                           "max_abs_diff_vs_plain": diff, "l2": l2}), flush=True)
 
 
-def long_context(partition_size: int = 0):
+def _profile_launches(fn, what: str, n: int = 3):
+    """n plain launches of fn for a profiler to capture; nothing is timed."""
+    for _ in range(n):
+        fn()
+    torch.cuda.synchronize()
+    _check()
+    print(json.dumps({"profile_launches": n, "workload": what}), flush=True)
+
+
+def long_context(partition_size: int = 0, profile: bool = False):
     S, H, D, CTX = 8, 32, 128, 32768
     lens, tables, nb = syn.long_context_tables(0, S, CTX)
     kp = torch.empty((nb, H, 16, D), dtype=torch.float16, device="cuda")
@@ -218,8 +230,12 @@ def long_context(partition_size: int = 0):
                      dtype=torch.uint8, device="cuda")
     out = torch.empty_like(q)
     pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=partition_size)
-    ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
-        pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size), 30)
+    run = lambda: pa.pa_decode_append_attention_planned(  # noqa: E731
+        pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size)
+    if profile:
+        _profile_launches(run, "long context: 8 x 32768 tokens, planned append + attend")
+        return
+    ms = _events_ms(run, 30)
     _check()
     kv_bytes = int(lens.sum()) * H * D * 2 * 2
     print(json.dumps({"kernel": "decode (long context)", "sequences": S, "context": CTX,
@@ -227,7 +243,7 @@ def long_context(partition_size: int = 0):
                       "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
-def single_layer():
+def single_layer(profile: bool = False):
     """One layer of 64 sequences, lengths uniform in [1, 2048], 32 heads x 128
     fp16, the pool exactly the used blocks at random places; the new token is
     appended and attended in one launch (about 1.1 GB of K/V, larger than L2)."""
@@ -245,8 +261,12 @@ def single_layer():
     ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
                      device="cuda")
     out = torch.empty_like(q)
-    ms = _events_ms(lambda: pa.pa_decode_append_attention(
-        pool, q, kn, vn, kp, vp, bt, cl, 1 / math.sqrt(D), out, ws), 50)
+    run = lambda: pa.pa_decode_append_attention(  # noqa: E731
+        pool, q, kn, vn, kp, vp, bt, cl, 1 / math.sqrt(D), out, ws)
+    if profile:
+        _profile_launches(run, "single layer: 64 sequences, plan + append + attend")
+        return
+    ms = _events_ms(run, 50)
     _check()
     kv_bytes = int(lens.sum()) * H * D * 2 * 2
     print(json.dumps({"kernel": "decode (single layer, plan + append + attend)", "sequences": S,
@@ -254,7 +274,7 @@ def single_layer():
                       "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
-def cache_ops():
+def cache_ops(profile: bool = False):
     """reshape_and_cache and copy_blocks at the sizes of the workloads: one
     decode step's new tokens (200), a long fill (32 768 tokens), and the
     copy-on-write of config 3 (127 block pairs); 32 heads x 128 fp16."""
@@ -270,6 +290,10 @@ def cache_ops():
         slots = torch.from_numpy(rng.permutation(nb * 16)[:T].astype(np.int32)).cuda()
         kn = torch.randn((T, H, D), dtype=torch.float16, device="cuda")
         vn = torch.randn_like(kn)
+        if profile:
+            _profile_launches(lambda: pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp),
+                              f"reshape_and_cache, {T} tokens", n=1)
+            continue
         us = _graph_us(lambda: pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp),
                        launches=50 if T <= 1024 else 5)
         _check()
@@ -278,6 +302,10 @@ def cache_ops():
                           "bytes_moved": moved, "GBps": round(moved / us / 1e3, 1)}), flush=True)
     perm = rng.permutation(nb)[:254].astype(np.int32)
     pairs = torch.from_numpy(perm.reshape(127, 2)).cuda()
+    if profile:
+        _profile_launches(lambda: pa.pa_copy_blocks(pool, kp, vp, pairs), "copy_blocks, 127 pairs",
+                          n=1)
+        return
     us = _graph_us(lambda: pa.pa_copy_blocks(pool, kp, vp, pairs))
     _check()
     moved = 2 * 2 * 127 * H * 16 * D * 2  # K and V blocks, read + written
@@ -328,8 +356,11 @@ def main(argv=None):
     sub.add_parser("shared-prefix")
     p = sub.add_parser("long-context")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
-    sub.add_parser("single-layer")
-    sub.add_parser("cache-ops")
+    p.add_argument("--profile", action="store_true")
+    p = sub.add_parser("single-layer")
+    p.add_argument("--profile", action="store_true")
+    p = sub.add_parser("cache-ops")
+    p.add_argument("--profile", action="store_true")
     sub.add_parser("decode-dtypes")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
@@ -342,11 +373,11 @@ def main(argv=None):
     elif args.what == "shared-prefix":
         shared_prefix()
     elif args.what == "long-context":
-        long_context(args.partition_size)
+        long_context(args.partition_size, args.profile)
     elif args.what == "single-layer":
-        single_layer()
+        single_layer(args.profile)
     elif args.what == "cache-ops":
-        cache_ops()
+        cache_ops(args.profile)
     else:
         decode_dtypes()
 

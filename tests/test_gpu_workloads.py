@@ -182,11 +182,26 @@ def test_long_context_split_k():
         assert np.array_equal(bits(kp[b, :, o]), bits(kn[s]))
 
 
-def test_full_decode_step_sampled():
+@pytest.mark.parametrize("path", ["fused-planned", "separate"])
+def test_full_decode_step_sampled(path):
     """200 requests x 32 layers x 32 heads x 128 fp16, one block-id space for
-    every layer; per layer reshape_and_cache of the new token then decode,
-    launched exactly as the benchmark launches them.  Layers 0 and 31 and
-    eight sequences are checked against the oracle."""
+    every layer (lengths min(2048, 1 + Exponential(500)), seed 0).
+
+    path "fused-planned" is the call sequence the benchmark times, launched
+    the same way: pa_decode_plan once for the step, then per layer one
+    pa_decode_append_attention_planned (the new token's reshape_and_cache and
+    the attention in one launch) with the automatic partition size (512
+    tokens at this batch) on the persistent grid, the plan reused by all 32
+    layers.  path "separate" runs pa_reshape_and_cache then
+    pa_decode_attention per layer.
+
+    For layers 0 and 31: both whole pools after the call are bit-identical to
+    the oracle's reshape_and_cache applied to host copies taken before it
+    ("Atención paginada en modelos de lenguaje grandes (LLM)", 7minutos.es,
+    section 2: the new token goes into the sequence's tail page), and the
+    outputs of nine sequences, the longest (split into partitions) among
+    them, match the oracle ("PagedAttention" wiki mirror, "Formulació
+    matemàtica")."""
     S, H, D, LAYERS = 200, 32, 128, 32
     lens = syn.full_step_lengths(seed=0, num_seqs=S)
     tables, nb = syn.full_step_tables(0, lens)
@@ -196,7 +211,15 @@ def test_full_decode_step_sampled():
     ws = workspace_for(pool, S, tables.shape[1])
     rng = np.random.default_rng(0)
     sample_layers = [0, LAYERS - 1]
-    sample_seqs = sorted(rng.choice(S, 8, replace=False).tolist())
+    longest = int(np.argmax(lens))
+    assert lens[longest] > 512  # split into several partitions
+    sample_seqs = sorted(set(rng.choice(S, 8, replace=False).tolist()) | {longest})
+    oslots = np.array([oracle.slot_of_c(tables[s], int(lens[s]) - 1) for s in range(S)],
+                      dtype=np.int32)
+    scale = 1 / math.sqrt(D)
+    fused = path == "fused-planned"
+    if fused:
+        pa.pa_decode_plan(pool, cld, tables.shape[1], ws)
     checked = 0
     for layer in range(LAYERS):
         kp = torch.empty((nb, H, BS, D), dtype=torch.float16, device="cuda")
@@ -210,18 +233,22 @@ def test_full_decode_step_sampled():
         if layer in sample_layers:
             kh, vh = host(kp), host(vp)
         out = torch.empty_like(q)
-        pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp)
-        pa.pa_decode_attention(pool, q, kp, vp, btd, cld, 1 / math.sqrt(D), out, ws)
+        if fused:
+            pa.pa_decode_append_attention_planned(pool, q, kn, vn, kp, vp, btd, scale, out, ws)
+        else:
+            pa.pa_reshape_and_cache(pool, kn, vn, slots, kp, vp)
+            pa.pa_decode_attention(pool, q, kp, vp, btd, cld, scale, out, ws)
         assert pa.pa_device_errors() == 0
         if layer in sample_layers:
-            oslots = np.array([oracle.slot_of_c(tables[s], int(lens[s]) - 1) for s in range(S)],
-                              dtype=np.int32)
             oracle.reshape_and_cache(host(kn), host(vn), oslots, kh, vh)
+            assert np.array_equal(bits(kp), bits(kh)), f"layer {layer}: K pool"
+            assert np.array_equal(bits(vp), bits(vh)), f"layer {layer}: V pool"
             only = np.zeros(S, dtype=np.int32)
             only[sample_seqs] = lens[sample_seqs]
-            ref = oracle.decode_attention(host(q), kh, vh, tables, only, 1 / math.sqrt(D))
-            assert_parity(out[sample_seqs], ref[sample_seqs], f"layer {layer}")
+            ref = oracle.decode_attention(host(q), kh, vh, tables, only, scale)
+            assert_parity(out[sample_seqs], ref[sample_seqs], f"{path}, layer {layer}")
             checked += 1
+            del kh, vh
         del kp, vp
     assert checked == len(sample_layers)
 
