@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 CU_SOURCES = ["pagedattn.cu"]
 CPP_SOURCES = ["block_manager.cpp", "status.cpp"]
 HEADERS = ["device_utils.cuh", "plan.cuh", "decode.cuh", "cache_ops.cuh", "status.h", "mma_utils.cuh",
-           "shared_prefix.cuh", "decode_gqa.cuh", "prefill.cuh"]
+           "shared_prefix.cuh", "decode_gqa.cuh", "prefill.cuh", "tma.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -10,13 +10,17 @@
 // precision); fp16 weights go in as they are.  The running max only moves,
 // and the accumulators are only rescaled, when a score passes it by more than
 // 2^8, so the rescale is rare and the weights stay at most 256.  The pipeline
-// is the MHA kernel's: a per-warp NSTAGE ring fed by
-// 1-D bulk copies on mbarriers, items from the plan's queue, split-K partials
-// merged by the last CTA to finish a sequence, optional fused append.  Rows
-// land in shared memory padded to D*2+16 bytes (one bulk copy per token row,
-// issued by 16 lanes for K and 16 for V), so ldmatrix reads are free of bank
-// conflicts; rows past the end of a ragged block are zero-filled instead of
-// copied, so stale pool contents never reach the product.
+// is the MHA kernel's: a per-warp NSTAGE ring on mbarriers, items from the
+// plan's queue, split-K partials merged by the last CTA to finish a
+// sequence, optional fused append.
+// Staging: each (block, KV head) tile of K and of V arrives whole, as D/64
+// tiled tensor copies of one 16-row x 128-byte box each (the pool viewed as
+// [blocks * heads * 16 rows][head_dim]), written with 128-byte swizzle so the
+// ldmatrix reads of the products are free of bank conflicts.  Four copies per
+// block at head_dim 128, issued by one lane.  V rows past the end of a ragged
+// block (stale, possibly NaN) are zeroed in shared memory after they land,
+// so they never reach the product; K rows there only produce scores that are
+// masked out.
 #pragma once
 
 #include <math.h>
@@ -27,6 +31,7 @@
 #include "decode.cuh"
 #include "device_utils.cuh"
 #include "mma_utils.cuh"
+#include "tma.cuh"
 
 namespace pa {
 
@@ -40,23 +45,32 @@ struct GqaConfig {
   static_assert(WARPS >= 1 && WARPS <= 4, "warps per CTA");
   static constexpr int THREADS = WARPS * 32;
   static constexpr int ROW_BYTES = D * 2;
-  static constexpr int PITCH = ROW_BYTES + 16;
-  static constexpr int TILE_BYTES = kBlock * PITCH;
+  static constexpr int BOXES = D / 64;              // 64-wide slices of head_dim
+  static constexpr int BOX_BYTES = kBlock * 128;    // 16 rows x 128 bytes, swizzled
+  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
+  static_assert(BOX_BYTES % 1024 == 0, "swizzled boxes start 1024-byte aligned");
+  // 1 KB of slack to align the stages, the stages, one mbarrier per stage,
+  // and the item's block-table slice
   static size_t smem_bytes(int partition_size) {
-    return (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
+    return 1024 + (size_t)WARPS * NSTAGE * STAGE_BYTES + (size_t)WARPS * NSTAGE * 8 +
            (size_t)(partition_size / kBlock) * 4;
   }
 };
 
+// tm_k, tm_v: the K and V pools as [num_blocks * heads * 16 rows][head_dim],
+// box {64, 16}, 128-byte swizzle.
 template <typename T, int D, int NSTAGE>
-__global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(128)
+    paged_decode_gqa_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v) {
   using Cfg = GqaConfig<T, D, NSTAGE>;
   constexpr int KSTEPS = D / 16;
   constexpr int NT = D / 8;
   constexpr int WARPS = Cfg::WARPS;
 
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t gqa_smem[];
+  uint8_t* smem = gqa_smem + ((1024u - (smem_addr(gqa_smem) & 1023u)) & 1023u);
   uint8_t* stages = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * NSTAGE * Cfg::STAGE_BYTES);
   int32_t* tbl = reinterpret_cast<int32_t*>(bars + WARPS * NSTAGE);
@@ -146,35 +160,29 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
 #pragma unroll
       for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
 
-      const char* kbase = static_cast<const char*>(a.k_pool) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
-      const char* vbase = static_cast<const char*>(a.v_pool) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
+      char* kbase = static_cast<char*>(const_cast<void*>(a.k_pool)) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
+      char* vbase = static_cast<char*>(const_cast<void*>(a.v_pool)) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
       const int64_t block_bytes = (int64_t)HK * kBlock * Cfg::ROW_BYTES;
-      // fill stage k with block bi: lanes 0-15 take K rows, 16-31 V rows; rows
-      // past the valid count are zeroed rather than copied
+      // fill stage k with block bi: lane 0 issues the tile copies of K and V
+      // (the host keeps every row coordinate below 2^31)
       auto issue = [&](uint32_t k, int bi) {
         const int st = k % NSTAGE;
         const uint32_t bar = smem_addr(&my_bars[st]);
-        uint8_t* dst = my_stages + st * Cfg::STAGE_BYTES;
-        const int valid = min(kBlock, ntok - bi * kBlock);
-        const int row = lane & 15;
-        const bool is_v = lane >= 16;
-        fence_proxy_async_shared();
-        if (lane == 0) mbar_arrive_expect_tx(bar, 2 * valid * Cfg::ROW_BYTES);
-        __syncwarp();
-        uint8_t* rdst = dst + (is_v ? Cfg::TILE_BYTES : 0) + row * Cfg::PITCH;
-        if (row < valid) {
-          const char* src = (is_v ? vbase : kbase) + (int64_t)tbl[bi] * block_bytes +
-                            (int64_t)row * Cfg::ROW_BYTES;
-          bulk_copy_g2s(smem_addr(rdst), src, Cfg::ROW_BYTES, bar);
-        } else {
+        const uint32_t dst = smem_addr(my_stages + st * Cfg::STAGE_BYTES);
+        const int y = (tbl[bi] * HK + kvh) * kBlock;
+        fence_proxy_async_shared();  // this lane ordered the warp's reads of the stage (syncwarp)
+        mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
 #pragma unroll
-          for (int c = 0; c < Cfg::ROW_BYTES / 16; ++c)
-            reinterpret_cast<uint4*>(rdst)[c] = make_uint4(0, 0, 0, 0);
+        for (int b = 0; b < Cfg::BOXES; ++b) {
+          tma_load_2d(dst + b * Cfg::BOX_BYTES, &tm_k, b * 64, y, bar);
+          tma_load_2d(dst + Cfg::TILE_BYTES + b * Cfg::BOX_BYTES, &tm_v, b * 64, y, bar);
         }
       };
 
       const uint32_t k0 = fills;
-      for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
+      __syncwarp();  // every lane is done with the previous item's stages
+      if (lane == 0)
+        for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
       bool ok = true;
       int i = 0;
       for (; i < nblk; ++i) {
@@ -185,34 +193,44 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
           ok = false;
           break;
         }
-        __syncwarp();  // the zero-filled rows of this stage are visible to every lane
         uint8_t* ktile = my_stages + st * Cfg::STAGE_BYTES;
         uint8_t* vtile = ktile + Cfg::TILE_BYTES;
         const int valid = min(kBlock, ntok - i * kBlock);
-        if (append && i == nblk - 1) {
-          // fused reshape_and_cache of the KV head's new row
-          if (lane < Cfg::ROW_BYTES / 16) {
-            const int64_t skv = (int64_t)s * HK + kvh;
-            const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + skv * D)[lane];
-            const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + skv * D)[lane];
-            reinterpret_cast<uint4*>(ktile + new_row * Cfg::PITCH)[lane] = kn;
-            reinterpret_cast<uint4*>(vtile + new_row * Cfg::PITCH)[lane] = vn;
-            const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * Cfg::ROW_BYTES;
-            reinterpret_cast<uint4*>(const_cast<char*>(kbase) + row_off)[lane] = kn;
-            reinterpret_cast<uint4*>(const_cast<char*>(vbase) + row_off)[lane] = vn;
+        if (valid < kBlock) {
+          // V rows past the context hold stale values (maybe NaN): zero them
+          // so that 0-weight x stale never reaches P.V
+          constexpr int CH = Cfg::BOXES * 8;  // 16-byte chunks per row
+          for (int c = lane; c < (kBlock - valid) * CH; c += 32) {
+            const int r = valid + c / CH;
+            *reinterpret_cast<uint4*>(vtile + (c % CH / 8) * Cfg::BOX_BYTES + r * 128 +
+                                      (c % 8) * 16) = make_uint4(0, 0, 0, 0);
           }
-          __syncwarp();
         }
+        if (append && i == nblk - 1 && lane < Cfg::ROW_BYTES / 16) {
+          // fused reshape_and_cache of the KV head's new row: into the pool,
+          // and over the stale row of the staged tiles
+          const int64_t skv = (int64_t)s * HK + kvh;
+          const uint4 kn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k_new) + skv * D)[lane];
+          const uint4 vn = reinterpret_cast<const uint4*>(static_cast<const T*>(a.v_new) + skv * D)[lane];
+          const uint32_t off = (lane / 8) * Cfg::BOX_BYTES + sw128_off(new_row, lane % 8);
+          *reinterpret_cast<uint4*>(ktile + off) = kn;
+          *reinterpret_cast<uint4*>(vtile + off) = vn;
+          const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * Cfg::ROW_BYTES;
+          reinterpret_cast<uint4*>(kbase + row_off)[lane] = kn;
+          reinterpret_cast<uint4*>(vbase + row_off)[lane] = vn;
+        }
+        __syncwarp();  // zeroed and appended rows are visible to every lane
 
         // S = Q K^T: sc[0] tokens 0-7, sc[1] tokens 8-15 (rows 0-7 in c0,c1)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
           const int row = (lane & 7) + ((lane >> 4) << 3);
-          const int col8 = ((lane >> 3) & 1) * 8;
+          const int half = (lane >> 3) & 1;  // which 8-element half of the k-step
 #pragma unroll
           for (int ks = 0; ks < KSTEPS; ++ks) {
             uint32_t b[4];
-            ldmatrix_x4(b, smem_addr(ktile + row * Cfg::PITCH + (ks * 16 + col8) * 2));
+            const int c = ks * 2 + half;  // 16-byte chunk of the row
+            ldmatrix_x4(b, smem_addr(ktile + (c / 8) * Cfg::BOX_BYTES + sw128_off(row, c % 8)));
             mma16816<T>(sc[0], qa[ks], b[0], b[1]);
             mma16816<T>(sc[1], qa[ks], b[2], b[3]);
           }
@@ -258,11 +276,12 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
         }
         {
           const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
-          const int col = (lane >> 4) * 8;
+          const int hi = lane >> 4;  // which of the two 8-wide column tiles
 #pragma unroll
           for (int j = 0; j < NT; j += 2) {
             uint32_t b[4];
-            ldmatrix_x4_trans(b, smem_addr(vtile + row * Cfg::PITCH + (j * 8 + col) * 2));
+            const int c = j + hi;  // 16-byte chunk of the row
+            ldmatrix_x4_trans(b, smem_addr(vtile + (c / 8) * Cfg::BOX_BYTES + sw128_off(row, c % 8)));
             float d0[4] = {o[j][0], o[j][1], 0.f, 0.f};
             float d1[4] = {o[j + 1][0], o[j + 1][1], 0.f, 0.f};
             mma16816<T>(d0, pa_, b[0], b[1]);
@@ -277,8 +296,8 @@ __global__ void __launch_bounds__(128) paged_decode_gqa_kernel(DecodeArgs a) {
             o[j + 1][1] = d1[1];
           }
         }
-        __syncwarp();
-        if (i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
+        __syncwarp();  // every lane is done with this stage
+        if (lane == 0 && i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
       }
       if (!ok) {
         if (lane == 0) {  // as in the MHA kernel: report, stop, and poison the plan

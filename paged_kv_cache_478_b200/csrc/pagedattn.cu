@@ -135,7 +135,8 @@ size_t prefill_smem() {
 
 // K or V pool as a 2-D tensor [num_blocks * heads * 16 rows][head_dim] with a
 // {64, 16} box (one physical block, one 64-wide slice of head_dim) and
-// 128-byte swizzle: the prefill kernel's tile layout.
+// 128-byte swizzle: the tile layout of the prefill and grouped-query decode
+// kernels.
 pa_status encode_pool_map(const DeviceState& dev, CUtensorMap* map, const void* base,
                           const pa_pool* pool) {
   const cuuint64_t dims[2] = {(cuuint64_t)pool->head_dim,
@@ -150,7 +151,7 @@ pa_status encode_pool_map(const DeviceState& dev, CUtensorMap* map, const void* 
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[96];
-    std::snprintf(buf, sizeof buf, "prefill: cuTensorMapEncodeTiled failed (%d)", (int)r);
+    std::snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled (pool) failed (%d)", (int)r);
     return fail(PA_ERR_CUDA, buf);
   }
   return PA_OK;
@@ -204,11 +205,11 @@ cudaError_t set_gqa_attrs() {
 // dependent launch on the preceding kernel of the stream (the shared-prefix
 // kernel): its CTAs may start while that kernel runs, and wait for it only
 // before merging a sequence that has shared-prefix partials.
-template <typename K>
+template <typename K, typename... Extra>
 cudaError_t launch_decode_grid(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
-                               const DecodeArgs& a, bool overlap) {
+                               const DecodeArgs& a, bool overlap, const Extra&... extra) {
   if (!overlap) {
-    kernel<<<grid, threads, smem, stream>>>(a);
+    kernel<<<grid, threads, smem, stream>>>(a, extra...);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -221,12 +222,12 @@ cudaError_t launch_decode_grid(K kernel, int grid, int threads, size_t smem, cud
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a, extra...);
 }
 
 template <typename T, int D>
 cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t stream,
-                       bool overlap = false) {
+                       const CUtensorMap& tm_k, const CUtensorMap& tm_v, bool overlap = false) {
   using Cfg = GqaConfig<T, D, kGqaStages>;
   auto kernel = paged_decode_gqa_kernel<T, D, kGqaStages>;
   const size_t smem = Cfg::smem_bytes(a.partition_size);
@@ -236,7 +237,7 @@ cudaError_t launch_gqa(const DecodeArgs& a, const DeviceState& dev, cudaStream_t
   per_sm = std::max(per_sm, 1);
   const int64_t upper = (int64_t)a.num_seqs * a.max_parts * a.head_groups;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(upper, (int64_t)dev.num_sms * per_sm));
-  return launch_decode_grid(kernel, grid, Cfg::THREADS, smem, stream, a, overlap);
+  return launch_decode_grid(kernel, grid, Cfg::THREADS, smem, stream, a, overlap, tm_k, tm_v);
 }
 
 // Once per device, with that device current: resolve the error word's device
@@ -652,11 +653,23 @@ pa_status launch_run(const pa_pool* pool, const DecodeArgs& a, const DeviceState
                      cudaStream_t s, bool overlap = false) {
   cudaError_t e;
   if (use_gqa_mma(pool)) {
+    // the tensor-core kernel stages tiles by tensor copies whose row
+    // coordinate (block * heads + head) * 16 must fit int32; a pool past that
+    // would not fit in device memory at these head sizes anyway
+    if ((int64_t)pool->num_blocks * pool->heads * kBlock > INT32_MAX)
+      return fail(PA_ERR_UNSUPPORTED, "decode: pool rows exceed the tensor-copy coordinate range");
+    CUtensorMap tk, tv;
+    pa_status st;
+    if ((st = encode_pool_map(dev, &tk, a.k_pool, pool)) != PA_OK ||
+        (st = encode_pool_map(dev, &tv, a.v_pool, pool)) != PA_OK)
+      return st;
     switch (pool->dtype * 1000 + pool->head_dim) {
-      case PA_F16 * 1000 + 64: e = launch_gqa<__half, 64>(a, dev, s, overlap); break;
-      case PA_F16 * 1000 + 128: e = launch_gqa<__half, 128>(a, dev, s, overlap); break;
-      case PA_BF16 * 1000 + 64: e = launch_gqa<__nv_bfloat16, 64>(a, dev, s, overlap); break;
-      case PA_BF16 * 1000 + 128: e = launch_gqa<__nv_bfloat16, 128>(a, dev, s, overlap); break;
+      case PA_F16 * 1000 + 64: e = launch_gqa<__half, 64>(a, dev, s, tk, tv, overlap); break;
+      case PA_F16 * 1000 + 128: e = launch_gqa<__half, 128>(a, dev, s, tk, tv, overlap); break;
+      case PA_BF16 * 1000 + 64: e = launch_gqa<__nv_bfloat16, 64>(a, dev, s, tk, tv, overlap); break;
+      case PA_BF16 * 1000 + 128:
+        e = launch_gqa<__nv_bfloat16, 128>(a, dev, s, tk, tv, overlap);
+        break;
       default: return fail(PA_ERR_UNSUPPORTED, "decode: dtype/head_dim not built");
     }
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode launch");

@@ -50,6 +50,7 @@
 #include "device_utils.cuh"
 #include "mma_utils.cuh"
 #include "pagedattn.h"
+#include "tma.cuh"
 
 namespace pa {
 
@@ -239,17 +240,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 2-D tiled tensor copy global -> shared (no multicast), completing its bytes
-// on `bar`.  x is the innermost coordinate (elements), y the row.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
 // 3-D tiled tensor copy global -> shared (no multicast); x innermost.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             int z, uint32_t bar) {
@@ -300,13 +290,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-
-// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile whose
-// rows are 128 bytes (one K-block).  The TMA copies with 128-byte swizzle
-// produce the same placement for boxes that start 1024-byte aligned.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-}
 
 template <typename T>
 constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
