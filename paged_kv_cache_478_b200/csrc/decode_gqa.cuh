@@ -58,6 +58,107 @@ struct GqaConfig {
   }
 };
 
+// Merge the partitions of all G query heads of one KV head (query heads
+// sh0 .. sh0+G-1) with one warp: 32/G lanes per query head, each lane owning
+// D*G/32 output dimensions, so the G merges run side by side.  The partial
+// rows are staged through the warp's ring buffer `buf` by bulk copies, PC
+// partitions of every head per round (one copy per head and round, all in
+// flight at once), and the (m, l) pairs of a round are loaded while the
+// copies fly: a merge costs about one memory round trip per round instead
+// of one per partition.  Rounds complete on the ring's barriers as ring
+// fills (`fills` counts them).  Per element the arithmetic and its order are
+// those of merge_partitions (max over the partitions, then the weighted sums
+// in partition order), so the results are the same bits.  Returns false if
+// a copy did not land in time (nothing is written then).
+template <typename T, int D, int G, int NSTAGE, int BUF>
+__device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, int np, int lane,
+                                            uint8_t* buf, uint64_t* bars, uint32_t& fills) {
+  using C = Chunk<T>;
+  constexpr int LPH = 32 / G;        // lanes per query head
+  constexpr int DPL = D / LPH;       // output dimensions per lane
+  constexpr int ROW = D * 4;         // one partial row, fp32
+  constexpr int PC = BUF / (G * ROW);  // partitions per round
+  static_assert(DPL % C::N == 0, "a lane owns whole 16-byte output chunks");
+  static_assert(PC >= 1, "the ring holds one partition of every head");
+  const int j = lane / LPH;
+  const int64_t sh = sh0 + j;
+  const int d0 = (lane % LPH) * DPL;
+  const float2* ml = a.part_ml + sh * a.max_parts;
+
+  // one round: lane 0 copies partitions [p0, p0 + n) of every head into buf
+  auto issue = [&](int p0, int n, uint32_t k) {
+    __syncwarp();  // every lane is done reading buf
+    if (lane == 0) {
+      const uint32_t bar = smem_addr(&bars[k % NSTAGE]);
+      fence_proxy_async_shared();
+      fence_proxy_async_global();  // partials other CTAs wrote, seen through the arrival count
+      mbar_arrive_expect_tx(bar, (uint32_t)(G * n * ROW));
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        bulk_copy_g2s(smem_addr(buf + h * PC * ROW),
+                      a.part_acc + ((sh0 + h) * a.max_parts + p0) * D, (uint32_t)(n * ROW), bar);
+    }
+  };
+  int n0 = min(PC, np);
+  uint32_t k = fills++;
+  issue(0, n0, k);
+
+  // the max over the partitions while the first round flies: the head's LPH
+  // lanes read every LPH-th partition, then combine (max is exact)
+  float M = -INFINITY;
+  for (int p = lane % LPH; p < np; p += LPH) M = fmaxf(M, __ldcg(&ml[p]).x);
+#pragma unroll
+  for (int m = 1; m < LPH; m <<= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
+
+  float den = 0.f;
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  bool ok = true;
+  for (int p0 = 0; p0 < np; p0 += PC) {
+    const int n = min(PC, np - p0);
+    float2 v[PC];
+#pragma unroll
+    for (int p = 0; p < PC; ++p) v[p] = p < n ? __ldcg(&ml[p0 + p]) : make_float2(0.f, 0.f);
+    if (p0 > 0) {
+      k = fills++;
+      issue(p0, n, k);
+    }
+    if (!__all_sync(kFullMask, mbar_wait_bounded(smem_addr(&bars[k % NSTAGE]), (k / NSTAGE) & 1u))) {
+      ok = false;
+      break;
+    }
+#pragma unroll
+    for (int p = 0; p < PC; ++p) {
+      if (p < n) {
+        const float w = exp2f(v[p].x - M);
+        den = fmaf(v[p].y, w, den);
+        const float4* src = reinterpret_cast<const float4*>(buf + (j * PC + p) * ROW + d0 * 4);
+#pragma unroll
+        for (int e = 0; e < DPL; e += 4) {
+          const float4 x = src[e / 4];
+          acc[e] = fmaf(w, x.x, acc[e]);
+          acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
+          acc[e + 2] = fmaf(w, x.z, acc[e + 2]);
+          acc[e + 3] = fmaf(w, x.w, acc[e + 3]);
+        }
+      }
+    }
+  }
+  if (!ok) {
+    mbar_wait_bounded(smem_addr(&bars[k % NSTAGE]), (k / NSTAGE) & 1u);  // let the copies land
+    return false;
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] *= inv;
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D + d0);
+#pragma unroll
+  for (int c = 0; c < DPL / C::N; ++c) dst[c] = C::from_float(acc + c * C::N);
+  __syncwarp();  // buf is read before the ring's next fill
+  return true;
+}
+
 // tm_k, tm_v: the K and V pools as [num_blocks * heads * 16 rows][head_dim],
 // box {64, 16}, 128-byte swizzle.
 template <typename T, int D, int NSTAGE>
@@ -347,7 +448,18 @@ __global__ void __launch_bounds__(128)
       if (s_merge && kvh < HK) {
         if (np > ni) grid_dependency_wait();  // shared-prefix partials: see the MHA kernel
         __threadfence();
-        for (int j = 0; j < G; ++j) merge_partitions<T, D>(a, (int64_t)s * HQ + kvh * G + j, np, lane);
+        constexpr int BUF = NSTAGE * Cfg::STAGE_BYTES;
+        const bool merged =
+            G == 8 ? merge_group<T, D, 8, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
+                                                       my_stages, my_bars, fills)
+                   : merge_group<T, D, 4, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
+                                                       my_stages, my_bars, fills);
+        if (!merged && lane == 0) {  // as for a copy of the item: report, stop, poison the plan
+          atomicOr(a.err, PA_DEVERR_TIMEOUT);
+          s_abort = 1;
+          a.plan->poisoned = 1;
+          __threadfence();
+        }
       }
     }
     __syncthreads();
