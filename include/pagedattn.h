@@ -253,7 +253,9 @@ pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
  * result stays correct.
  * Workspace: pa_decode_shared_prefix_workspace_bytes (max_shared_blocks
  * extra slots per head).  pa_find_shared_prefixes builds groups from host
- * block tables.
+ * block tables.  partition_size 0 here means 256-token partitions: the
+ * decode kernel attends only each sequence's own tokens, typically far
+ * fewer than max_context_len.
  */
 pa_status pa_decode_shared_prefix_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
                                                   int32_t max_blocks_per_seq,

@@ -121,18 +121,22 @@ __device__ __forceinline__ void ring_sync(int r) {
 }
 
 // Merge the partitions of (sequence s, head h) by log-sum-exp, in partition
-// order, and write the normalised output.  Lanes < CPR each own one 16-byte
-// output chunk.  Partials are read with .cg loads (L2), since other CTAs
-// wrote them during this launch.
+// order, and write the normalised output.  The max over the partitions is
+// read by all 32 lanes at once (every 32nd partition each, then combined:
+// max is exact, so the split changes no bit); then lanes < CPR each own one
+// 16-byte output chunk.  Partials are read with .cg loads (L2), since other
+// CTAs wrote them during this launch.  Called by all 32 lanes of the warp.
 template <typename T, int D>
 __device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t sh, int np, int lane) {
   using C = Chunk<T>;
   constexpr int VEC = C::N;
   constexpr int CPR = D / VEC;
-  if (lane >= CPR) return;
   const float2* ml = a.part_ml + sh * a.max_parts;
   float M = -INFINITY;
-  for (int p = 0; p < np; ++p) M = fmaxf(M, __ldcg(&ml[p]).x);
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(&ml[p]).x);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
+  if (lane >= CPR) return;
   float den = 0.f;
   float acc[VEC];
 #pragma unroll
@@ -157,6 +161,92 @@ __device__ __forceinline__ void merge_partitions(const DecodeArgs& a, int64_t sh
 #pragma unroll
   for (int e = 0; e < VEC; ++e) acc[e] *= inv;
   reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D)[lane] = C::from_float(acc);
+}
+
+// Four or two consecutive output values of one lane, rounded like Chunk<T>.
+template <typename T, int N>
+__device__ __forceinline__ void store_out(T* dst, const float* v) {
+  if constexpr (sizeof(T) == 4) {
+    if constexpr (N == 4) *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+  } else {
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = e < N ? v[e] : 0.f;
+    const uint4 u = Chunk<T>::from_float(f);  // pairs rounded as in a full chunk
+    if constexpr (N == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(u.x, u.y);
+    else *reinterpret_cast<uint32_t*>(dst) = u.x;
+  }
+}
+
+// The merge of merge_partitions for a warp that owns a bulk-copy ring (one
+// query head per ring): the partial rows come into the ring buffer `buf` by
+// one bulk copy per round of up to BUF / (4 D) partitions, while the lanes
+// read the (m, l) pairs (one partition per lane) and the max; every lane then
+// owns D/32 output values.  About one memory round trip per round instead of
+// one per few partitions.  Rounds complete on the ring's barriers as ring
+// fills, the first being fill number `fill0`.  Per element the arithmetic and
+// its order are those of merge_partitions, so the results are the same bits.
+// Returns the number of fills used, negated if a copy did not land in time
+// (nothing is written then).
+template <typename T, int D, int NSTAGE, int BUF>
+__device__ __forceinline__ int merge_staged(const DecodeArgs& a, int64_t sh, int np, int lane,
+                                            uint8_t* buf, uint64_t* bars, uint32_t fill0) {
+  constexpr int ROW = D * 4;                        // one partial row, fp32
+  constexpr int PC = BUF / ROW < 32 ? BUF / ROW : 32;  // partitions per round
+  constexpr int DPL = D / 32;                        // output values per lane
+  static_assert(PC >= 1 && (DPL == 4 || DPL == 2), "merge layout");
+  const float2* ml = a.part_ml + sh * a.max_parts;
+  const float* acc_src = a.part_acc + sh * a.max_parts * D;
+  auto issue = [&](int p0, int n, uint32_t k) {
+    __syncwarp();  // every lane is done reading buf
+    if (lane == 0) {
+      const uint32_t bar = smem_addr(&bars[k % NSTAGE]);
+      fence_proxy_async_shared();
+      fence_proxy_async_global();  // partials other CTAs wrote, seen through the arrival count
+      mbar_arrive_expect_tx(bar, (uint32_t)(n * ROW));
+      bulk_copy_g2s(smem_addr(buf), acc_src + (int64_t)p0 * D, (uint32_t)(n * ROW), bar);
+    }
+  };
+  uint32_t k = fill0;
+  issue(0, min(PC, np), k);
+  float M = -INFINITY;
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(&ml[p]).x);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
+  float den = 0.f;
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  bool ok = true;
+  for (int p0 = 0; p0 < np; p0 += PC) {
+    const int n = min(PC, np - p0);
+    const float2 v = lane < n ? __ldcg(&ml[p0 + lane]) : make_float2(0.f, 0.f);
+    if (p0 > 0) issue(p0, n, ++k);
+    if (!__all_sync(kFullMask, mbar_wait_bounded(smem_addr(&bars[k % NSTAGE]), (k / NSTAGE) & 1u))) {
+      ok = false;
+      break;
+    }
+    for (int p = 0; p < n; ++p) {
+      const float vx = __shfl_sync(kFullMask, v.x, p), vy = __shfl_sync(kFullMask, v.y, p);
+      const float w = exp2f(vx - M);
+      den = fmaf(vy, w, den);
+      const float* src = reinterpret_cast<const float*>(buf + p * ROW) + lane * DPL;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+    }
+  }
+  const int used = (int)(k - fill0) + 1;
+  if (!ok) {
+    mbar_wait_bounded(smem_addr(&bars[k % NSTAGE]), (k / NSTAGE) & 1u);  // let the copy land
+    return -used;
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] *= inv;
+  store_out<T, DPL>(static_cast<T*>(a.out) + sh * D + lane * DPL, acc);
+  __syncwarp();  // buf is read before the ring's next fill
+  return used;
 }
 
 // The persistent partition kernel: CTAs pull (sequence, partition, head
@@ -413,7 +503,21 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
         // complete before reading them (returns at once otherwise)
         if (np > ni) grid_dependency_wait();
         __threadfence();
-        merge_partitions<T, D>(a, (int64_t)s * HQ + hq, np, lane);
+        if constexpr (G == 1) {
+          // one query head per ring: the partials come through the warp's ring
+          constexpr int BUF = NSTAGE * Cfg::STAGE_BYTES;
+          const int used =
+              merge_staged<T, D, NSTAGE, BUF>(a, (int64_t)s * HQ + hq, np, lane, my_stages, my_bars, fills);
+          fills += used > 0 ? used : -used;
+          if (used < 0 && lane == 0) {  // as for a copy of the item: report, stop, poison the plan
+            atomicOr(a.err, PA_DEVERR_TIMEOUT);
+            s_abort = 1;
+            a.plan->poisoned = 1;
+            __threadfence();
+          }
+        } else {
+          merge_partitions<T, D>(a, (int64_t)s * HQ + hq, np, lane);
+        }
       }
     }
     __syncthreads();

@@ -64,6 +64,13 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's view of global memory (including writes by other
+// threads that it has synchronised with) before its later async-proxy (bulk
+// copy) reads of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 1-D bulk copy global -> shared, completing `bytes` transactions on `bar`.
 // dst and src 16-byte aligned, bytes a multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,

@@ -147,22 +147,36 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
         continue;
       }
       const int32_t* rt = a.block_tables + (int64_t)rep * a.max_blocks_per_seq;
-      // one warp per member: its lanes compare 32 table entries at a time
+      // each warp takes MPW members at a time, their lanes comparing 32 table
+      // entries per step, with the loads of all MPW members in flight together
+      constexpr int MPW = 4;
       const int lane = threadIdx.x & 31;
-      for (int m = m0 + (threadIdx.x >> 5); m < m1; m += blockDim.x >> 5) {
-        const int s = a.group_members[m];
-        bool ok = s >= 0 && s < a.num_seqs && a.lens[s] >= nbk * kBlock;
-        if (ok) {
-          const int32_t* t = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-          int diff = 0;
-          for (int j = lane; j < nbk; j += 32) diff |= t[j] ^ rt[j];
-          ok = !__any_sync(kFullMask, diff != 0);
+      for (int mb = m0 + (threadIdx.x >> 5) * MPW; mb < m1; mb += (blockDim.x >> 5) * MPW) {
+        int sv[MPW], diff[MPW];
+        bool ok[MPW];
+#pragma unroll
+        for (int u = 0; u < MPW; ++u) sv[u] = mb + u < m1 ? a.group_members[mb + u] : -1;
+#pragma unroll
+        for (int u = 0; u < MPW; ++u) {
+          ok[u] = sv[u] >= 0 && sv[u] < a.num_seqs && a.lens[sv[u]] >= nbk * kBlock;
+          diff[u] = 0;
         }
-        if (lane == 0) {
-          if (!ok) {
-            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
-          } else if (atomicCAS(&a.shared_of[s], -1, g) != -1) {
-            atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
+        for (int j = lane; j < nbk; j += 32) {
+          const int32_t r = rt[j];
+#pragma unroll
+          for (int u = 0; u < MPW; ++u)
+            if (ok[u]) diff[u] |= a.block_tables[(int64_t)sv[u] * a.max_blocks_per_seq + j] ^ r;
+        }
+#pragma unroll
+        for (int u = 0; u < MPW; ++u) {
+          if (mb + u >= m1) break;  // the same for the whole warp
+          const bool good = ok[u] && !__any_sync(kFullMask, diff[u] != 0);
+          if (lane == 0) {
+            if (!good) {
+              atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);
+            } else if (atomicCAS(&a.shared_of[sv[u]], -1, g) != -1) {
+              atomicOr(a.err, PA_DEVERR_CONTEXT_LEN);  // already in another group
+            }
           }
         }
       }

@@ -20,13 +20,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Order this thread's view of global memory (including writes by other
-// threads that it has synchronised with) before its later async-proxy (bulk
-// copy) reads of global memory.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled tile whose
 // rows are 128 bytes (64 fp16/bf16 elements).  TMA copies with 128-byte
 // swizzle produce this placement for boxes that start 1024-byte aligned.

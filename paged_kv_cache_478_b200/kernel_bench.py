@@ -1,8 +1,8 @@
 """Per-kernel timings on synthetic workloads (CUDA events on the launching stream).
 
     python -m paged_kv_cache_478_b200.kernel_bench prefill [--small]
-    python -m paged_kv_cache_478_b200.kernel_bench gqa
-    python -m paged_kv_cache_478_b200.kernel_bench shared-prefix
+    python -m paged_kv_cache_478_b200.kernel_bench gqa [--groups 4,8] [--profile]
+    python -m paged_kv_cache_478_b200.kernel_bench shared-prefix [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench long-context [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench single-layer [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench cache-ops [--profile]
@@ -123,7 +123,7 @@ def prefill(small: bool):
 _DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
 
-def gqa(partition_size: int = 0, dtype: str = "f16"):
+def gqa(partition_size: int = 0, dtype: str = "f16", profile: bool = False, groups=(1, 2, 4, 8)):
     S, HK, D = 200, 8, 128
     dt = _DTYPES[dtype]
     elt = torch.tensor([], dtype=dt).element_size()
@@ -135,7 +135,7 @@ def gqa(partition_size: int = 0, dtype: str = "f16"):
     syn.fill_normal_device(vp, 2)
     bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
     kv_bytes = int(lens.sum()) * HK * D * elt * 2
-    for G in (1, 2, 4, 8):
+    for G in groups:
         pool = pa.pa_pool_create(nb, 16, HK, D, dt)
         pa.pa_pool_set_query_heads(pool, HK * G)
         q = torch.randn((S, HK * G, D), dtype=dt, device="cuda")
@@ -145,9 +145,12 @@ def gqa(partition_size: int = 0, dtype: str = "f16"):
         ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, partition_size),
                          dtype=torch.uint8, device="cuda")
         pa.pa_decode_plan(pool, cl, tables.shape[1], ws, partition_size=partition_size)
-        ms = _events_ms(lambda: pa.pa_decode_append_attention_planned(
-            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size),
-            50)
+        run = lambda: pa.pa_decode_append_attention_planned(  # noqa: E731
+            pool, q, kn, vn, kp, vp, bt, 1 / math.sqrt(D), out, ws, partition_size=partition_size)
+        if profile:
+            _profile_launches(run, f"GQA decode, {G} query heads per KV head")
+            continue
+        ms = _events_ms(run, 50)
         _check()
         print(json.dumps({"kernel": "decode (GQA)", "dtype": dtype, "q_per_kv": G, "kv_heads": HK,
                           "partition_size": partition_size or "auto",
@@ -155,7 +158,7 @@ def gqa(partition_size: int = 0, dtype: str = "f16"):
               flush=True)
 
 
-def shared_prefix():
+def shared_prefix(profile: bool = False):
     H, D, S, P = 32, 128, 128, 1000
     case = syn.shared_prefix_case(0)
     nb = 63 + S + sum(math.ceil(int(n) / 16) for n in case["suffix_lens"])
@@ -193,6 +196,9 @@ def shared_prefix():
     plain = lambda: pa.pa_decode_attention(pool, q, kp, vp, bt, cl, scale, out1, ws1)  # noqa: E731
     shared = lambda: pa.pa_decode_attention_shared_prefix(  # noqa: E731
         pool, q, kp, vp, bt, cl, gd, scale, out2, ws2)
+    if profile:
+        _profile_launches(shared, "shared-prefix path: plan + shared-prefix kernel + decode")
+        return
     rows = []
     for l2, fl in (("flushed before every rep", flush), ("warm", None)):
         rows.append(("plain decode", l2, _events_ms(plain, 50, flush=fl)))
@@ -353,7 +359,10 @@ def main(argv=None):
     p = sub.add_parser("gqa")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     p.add_argument("--dtype", choices=sorted(_DTYPES), default="f16")
-    sub.add_parser("shared-prefix")
+    p.add_argument("--profile", action="store_true")
+    p.add_argument("--groups", default="1,2,4,8", help="query heads per KV head to run")
+    p = sub.add_parser("shared-prefix")
+    p.add_argument("--profile", action="store_true")
     p = sub.add_parser("long-context")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     p.add_argument("--profile", action="store_true")
@@ -369,9 +378,10 @@ def main(argv=None):
     if args.what == "prefill":
         prefill(args.small)
     elif args.what == "gqa":
-        gqa(args.partition_size, args.dtype)
+        gqa(args.partition_size, args.dtype, args.profile,
+            tuple(int(g) for g in args.groups.split(",")))
     elif args.what == "shared-prefix":
-        shared_prefix()
+        shared_prefix(args.profile)
     elif args.what == "long-context":
         long_context(args.partition_size, args.profile)
     elif args.what == "single-layer":
