@@ -3,13 +3,12 @@
   * The reference arm times the CPU oracle on a bounded sample of the decode
     step and prints one JSON line with the keys the harness reads; ranks
     other than 0 print nothing.
-  * The roofline's DRAM traffic comes from the committed ncu summary of the
-    decode kernel and is reported only while that summary's recorded source
-    hash is the current kernel source's.
+  * The roofline's DRAM traffic comes from the committed record of the ncu
+    capture of the decode kernel and is reported only while the record's
+    hash of the kernel's device sources is the current one.
 """
 import json
 import os
-import re
 import subprocess
 import sys
 
@@ -50,11 +49,11 @@ def test_reference_arm_runs_on_rank_0_only():
 
 
 def test_traffic_is_reported_only_for_the_profiled_source(monkeypatch):
-    text = open(bench.TRAFFIC_FILE).read()
-    recorded_hash = re.search(r"decode\.cuh sha256\[:16\]: `([0-9a-f]{16})`", text).group(1)
-    recorded_bytes = float(re.search(r"dram bytes per launch \(read \+ write\): `(\d+)`",
-                                     text).group(1))
-    monkeypatch.setattr(bench, "decode_source_hash", lambda: recorded_hash)
-    assert bench.committed_traffic() == recorded_bytes
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    assert rec["sources"] == list(bench.DECODE_SOURCES)
+    assert rec["dram_bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    monkeypatch.setattr(bench, "decode_source_hash", lambda: rec["sources_sha256_16"])
+    assert bench.committed_traffic() == float(rec["dram_bytes_per_launch"])
     monkeypatch.setattr(bench, "decode_source_hash", lambda: "0" * 16)
     assert bench.committed_traffic() is None
+
