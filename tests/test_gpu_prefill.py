@@ -156,3 +156,49 @@ def test_prefill_skips_a_sequence_whose_rows_fall_outside_q():
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT_LEN
     assert torch.count_nonzero(out[32:]) == 0
     assert_parity(out[:32], c["ref"][:32], "the sequence inside q still runs")
+
+
+@pytest.mark.parametrize("kv_heads,group", [(32, 1), (8, 4)])
+def test_prefill_with_several_items_per_cta(kv_heads, group):
+    """fp16 runs one persistent CTA per SM, each walking several 256-query
+    items in turn, with the next item's first products overlapping the end of
+    the current one.  384 items here (32 query heads x 3 prompts x 4 pairs),
+    so every CTA takes two or three; sampled rows against the oracle,
+    including the first and last rows of each query tile."""
+    ctx = [(1500, 1024), (1100, 1024), (1024, 1000)]
+    rng = np.random.default_rng(90 + group)
+    S, D = len(ctx), 128
+    lens = np.array([c for c, _ in ctx], dtype=np.int32)
+    news = np.array([n for _, n in ctx], dtype=np.int32)
+    need = [math.ceil(int(L) / 16) for L in lens]
+    nb = sum(need) + 3
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((S, max(need)), -1, dtype=np.int32)
+    pos = 0
+    for s, n in enumerate(need):
+        tables[s, :n] = perm[pos:pos + n]
+        pos += n
+    kt = torch.from_numpy(rng.standard_normal((nb, kv_heads, 16, D)).astype(np.float32)).half()
+    vt = torch.from_numpy(rng.standard_normal((nb, kv_heads, 16, D)).astype(np.float32)).half()
+    T = int(news.sum())
+    qt = torch.from_numpy(rng.standard_normal((T, kv_heads * group, D)).astype(np.float32)).half()
+    qs = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
+    pool = pa.pa_pool_create(nb, 16, kv_heads, D, torch.float16)
+    pa.pa_pool_set_query_heads(pool, kv_heads * group)
+    out = torch.empty_like(qt.cuda())
+    scale = 1 / math.sqrt(D)
+    pa.pa_prefill_attention(pool, qt.cuda(), kt.cuda(), vt.cuda(), dev(tables), dev(lens), dev(qs),
+                            scale, out, int(news.max()))
+    assert pa.pa_device_errors() == 0
+    rows, row_t, row_l = [], [], []
+    for s in range(S):
+        n = int(news[s])
+        pick = {0, 127, 128, 255, 256, 511, 512, n - 1}
+        pick |= set(rng.choice(n, 24, replace=False).tolist())
+        for i in sorted(p for p in pick if p < n):
+            rows.append(int(qs[s]) + i)
+            row_t.append(tables[s])
+            row_l.append(int(lens[s]) - n + i + 1)
+    ref = oracle.decode_attention(qt.numpy()[rows], kt.numpy(), vt.numpy(), np.stack(row_t),
+                                  np.array(row_l, np.int32), scale)
+    assert_parity(out[rows], ref, f"prefill, several items per CTA, G={group}")
