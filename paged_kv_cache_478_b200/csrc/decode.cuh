@@ -24,9 +24,10 @@
 //   * fp32 online softmax in the log2 domain (q is pre-scaled by
 //     scale*log2(e)); P.V accumulates in fp32 registers.
 //   * Work items are handed out by an atomic counter in the workspace, in the
-//     order a one-CTA plan kernel wrote: full partitions first, then the
-//     ragged last partitions by decreasing size, so the tail of the grid is
-//     made of the smallest items.
+//     order a one-CTA plan kernel wrote: the ragged last partitions of split
+//     sequences, the full partitions, then the unsplit sequences by
+//     decreasing size, so the merges fall mid-launch and the tail of the
+//     grid is made of the smallest items, which merge nothing.
 //   * Sequences with more than one partition write (m, l, unnormalised acc)
 //     per partition and bump a per-(sequence, head group) arrival counter;
 //     the CTA that arrives last merges all partitions by log-sum-exp in

@@ -660,7 +660,7 @@ pa_status check_plan(const pa_pool* pool, DecodeArgs* a, const char* who) {
 // follow in the same call) and record it for the workspace.
 pa_status launch_plan(const pa_pool* pool, DecodeArgs* a, cudaStream_t s) {
   a->stamp = next_plan_stamp();
-  decode_plan_kernel<<<1, 1024, (a->partition_size / kBlock + 1) * sizeof(int32_t), s>>>(*a);
+  decode_plan_kernel<<<1, 1024, 2 * (a->partition_size / kBlock + 1) * sizeof(int32_t), s>>>(*a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode plan launch");
   const PlanKey k = plan_key(pool, *a);

@@ -2,8 +2,12 @@
 //
 // The plan kernel (one CTA per call, or once per step with the planned API)
 // validates context lengths and shared-prefix groups and orders the work
-// items the decode kernels take from an atomic queue: full partitions first,
-// then the ragged last partitions by decreasing size.  It lives apart from
+// items the decode kernels take from an atomic queue: the ragged last
+// partitions of split sequences first (by decreasing size), then the full
+// partitions, then the sequences that fit one partition (by decreasing
+// size).  A split sequence is merged when its last partition arrives, so
+// this puts the merges in the middle of the launch instead of at its end,
+// and leaves the tail to unsplit items, which merge nothing.  It lives apart from
 // the decode kernel so that the decode kernel's source (whose DRAM traffic
 // profiles record) changes only with the kernel.
 #pragma once
@@ -108,12 +112,17 @@ __device__ __forceinline__ bool plan_item(const DecodeArgs& a, int item, PlanIte
 // ---- plan: one CTA orders the work ------------------------------------------------
 
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
-  extern __shared__ int32_t bucket[];  // [nb + 1]: index 0 = sequences with no own tokens
-  __shared__ int32_t n_full;
+  // bucket[0..nb]: ragged last partitions of split sequences by block count;
+  // bucket[nb+1..2nb+1]: unsplit sequences by block count (nb+1: no own tokens)
+  extern __shared__ int32_t bucket[];
+  __shared__ int32_t n_full, n_full2, full_base;  // full partitions: count, placed, first slot
   const int PS = a.partition_size;
   const int nb = PS / kBlock;
-  for (int i = threadIdx.x; i <= nb; i += blockDim.x) bucket[i] = 0;
-  if (threadIdx.x == 0) n_full = 0;
+  for (int i = threadIdx.x; i <= 2 * nb + 1; i += blockDim.x) bucket[i] = 0;
+  if (threadIdx.x == 0) {
+    n_full = 0;
+    n_full2 = 0;
+  }
   const int cap = (int)min((int64_t)a.max_context_len, (int64_t)a.max_blocks_per_seq * kBlock);
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     int L = a.context_lens[s];
@@ -194,16 +203,21 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
     a.base[s] = base;
     a.nitems[s] = ni;
     a.nparts[s] = ni + (sb > 0 ? (sb + a.shared_chunk - 1) / a.shared_chunk : 0);
-    if (full > 0) {
-      const int pos = atomicAdd(&n_full, full);
-      for (int p = 0; p < full; ++p) a.pairs[pos + p] = make_int2(s, p);
-    }
-    if (U == 0 || rem > 0) atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
+    if (full > 0) atomicAdd(&n_full, full);
+    if (U == 0 || rem > 0)  // a ragged last partition, or the whole (possibly empty) sequence
+      atomicAdd(&bucket[(full > 0 ? 0 : nb + 1) + (U == 0 ? 0 : (rem + kBlock - 1) / kBlock)], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int run = n_full;
-    for (int b = nb; b >= 0; --b) {  // biggest remainders first, empty ones last
+    int run = 0;
+    for (int b = nb; b >= 0; --b) {  // remainders of split sequences, biggest first
+      const int c = bucket[b];
+      bucket[b] = run;
+      run += c;
+    }
+    full_base = run;  // then the full partitions
+    run += n_full;
+    for (int b = 2 * nb + 1; b > nb; --b) {  // then the unsplit sequences, biggest first
       const int c = bucket[b];
       bucket[b] = run;
       run += c;
@@ -218,10 +232,15 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int U = a.lens[s] - a.base[s];
-    const int rem = U % PS;
+    const int rem = U % PS, full = U / PS;
+    if (full > 0) {
+      const int pos = full_base + atomicAdd(&n_full2, full);
+      for (int p = 0; p < full; ++p) a.pairs[pos + p] = make_int2(s, p);
+    }
     if (U == 0 || rem > 0) {
-      const int pos = atomicAdd(&bucket[U == 0 ? 0 : (rem + kBlock - 1) / kBlock], 1);
-      a.pairs[pos] = make_int2(s, U / PS);
+      const int b = (full > 0 ? 0 : nb + 1) + (U == 0 ? 0 : (rem + kBlock - 1) / kBlock);
+      const int pos = atomicAdd(&bucket[b], 1);
+      a.pairs[pos] = make_int2(s, full);
     }
   }
 }
