@@ -78,7 +78,7 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
   constexpr int DPL = D / LPH;       // output dimensions per lane
   constexpr int ROW = D * 4;         // one partial row, fp32
   constexpr int PC = BUF / (G * ROW);  // partitions per round
-  static_assert(DPL % C::N == 0, "a lane owns whole 16-byte output chunks");
+  static_assert(DPL % C::N == 0 || DPL == 4, "a lane owns whole 16-byte output chunks");
   static_assert(PC >= 1, "the ring holds one partition of every head");
   const int j = lane / LPH;
   const int64_t sh = sh0 + j;
@@ -152,9 +152,13 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
   const float inv = 1.f / den;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] *= inv;
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D + d0);
+  if constexpr (DPL % C::N == 0) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D + d0);
 #pragma unroll
-  for (int c = 0; c < DPL / C::N; ++c) dst[c] = C::from_float(acc + c * C::N);
+    for (int c = 0; c < DPL / C::N; ++c) dst[c] = C::from_float(acc + c * C::N);
+  } else {
+    store_out<T, DPL>(static_cast<T*>(a.out) + sh * D + d0, acc);
+  }
   __syncwarp();  // buf is read before the ring's next fill
   return true;
 }
@@ -450,10 +454,12 @@ __global__ void __launch_bounds__(128)
         __threadfence();
         constexpr int BUF = NSTAGE * Cfg::STAGE_BYTES;
         const bool merged =
-            G == 8 ? merge_group<T, D, 8, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
-                                                       my_stages, my_bars, fills)
-                   : merge_group<T, D, 4, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
-                                                       my_stages, my_bars, fills);
+            G == 8   ? merge_group<T, D, 8, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
+                                                         my_stages, my_bars, fills)
+            : G == 4 ? merge_group<T, D, 4, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
+                                                         my_stages, my_bars, fills)
+                     : merge_group<T, D, 2, NSTAGE, BUF>(a, (int64_t)s * HQ + kvh * G, np, lane,
+                                                         my_stages, my_bars, fills);
         if (!merged && lane == 0) {  // as for a copy of the item: report, stop, poison the plan
           atomicOr(a.err, PA_DEVERR_TIMEOUT);
           s_abort = 1;

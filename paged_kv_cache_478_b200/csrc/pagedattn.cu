@@ -115,10 +115,12 @@ cudaError_t set_decode_attrs_all_groups() {
 // KV heads one work item covers, for G query heads per KV head.
 int rings_for(int G) { return warps_for(G) / G; }
 
-// Groups of 4 or 8 query heads on fp16/bf16 pools take the tensor-core
-// kernel (one warp per KV head); MHA, pairs (measured faster on CUDA cores)
-// and fp32 pools take the CUDA-core kernel.
-bool use_gqa_mma(const pa_pool* pool) { return pool->q_per_kv >= 4 && pool->dtype != PA_F32; }
+// Groups of 2, 4 or 8 query heads on fp16/bf16 pools take the tensor-core
+// kernel (one warp per KV head); MHA and fp32 pools take the CUDA-core
+// kernel.  (Pairs once ran faster on CUDA cores; since the tensor-core
+// kernel stages whole tiles and merges all heads of a KV head at once it
+// is faster for them too: 106 -> 89 us on 200 requests x 8 KV heads.)
+bool use_gqa_mma(const pa_pool* pool) { return pool->q_per_kv >= 2 && pool->dtype != PA_F32; }
 #ifndef PA_GQA_STAGES
 #define PA_GQA_STAGES 2
 #endif

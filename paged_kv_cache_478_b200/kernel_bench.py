@@ -1,6 +1,6 @@
 """Per-kernel timings on synthetic workloads (CUDA events on the launching stream).
 
-    python -m paged_kv_cache_478_b200.kernel_bench prefill [--small]
+    python -m paged_kv_cache_478_b200.kernel_bench prefill [--small | --profile]
     python -m paged_kv_cache_478_b200.kernel_bench gqa [--groups 4,8] [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench shared-prefix [--profile]
     python -m paged_kv_cache_478_b200.kernel_bench long-context [--profile]
@@ -101,7 +101,7 @@ def _prefill_case(seqs, new_tokens, kv_heads, group, head_dim, dtype, seed=0):
     return run, flops
 
 
-def prefill(small: bool):
+def prefill(small: bool, profile: bool = False):
     if small:
         run, _ = _prefill_case(2, 2048, 32, 1, 128, torch.float16)
         for _ in range(3):
@@ -109,6 +109,10 @@ def prefill(small: bool):
         torch.cuda.synchronize()
         _check()
         print(json.dumps({"prefill_small_case": "2 x 2048 fp16, 32 heads x 128, 3 launches"}))
+        return
+    if profile:
+        run, _ = _prefill_case(4, 4096, 32, 1, 128, torch.float16)
+        _profile_launches(run, "prefill, 4 prompts x 4096 fp16, 32 heads x 128")
         return
     for seqs, n, hk, g, dt in [(4, 4096, 32, 1, torch.float16), (8, 2048, 32, 1, torch.float16),
                                (16, 1024, 8, 4, torch.float16), (8, 2048, 32, 1, torch.bfloat16)]:
@@ -356,6 +360,7 @@ def main(argv=None):
     sub = ap.add_subparsers(dest="what", required=True)
     p = sub.add_parser("prefill")
     p.add_argument("--small", action="store_true", help="3 launches of 2 x 2048 fp16 (profiling)")
+    p.add_argument("--profile", action="store_true", help="3 launches of 4 x 4096 fp16 (profiling)")
     p = sub.add_parser("gqa")
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     p.add_argument("--dtype", choices=sorted(_DTYPES), default="f16")
@@ -376,7 +381,7 @@ def main(argv=None):
         raise SystemExit("kernel_bench needs a CUDA device")
     torch.manual_seed(0)  # the q tensors drawn below are the same in every run
     if args.what == "prefill":
-        prefill(args.small)
+        prefill(args.small, args.profile)
     elif args.what == "gqa":
         gqa(args.partition_size, args.dtype, args.profile,
             tuple(int(g) for g in args.groups.split(",")))
