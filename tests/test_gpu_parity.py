@@ -429,7 +429,7 @@ def test_gqa_matches_oracle_and_replicated_mha(group, dtype, head_dim):
         assert_parity(out, out_r.double().cpu().numpy(), f"gqa x{group} vs repeated-KV MHA")
 
 
-@pytest.mark.parametrize("group", [4, 8])
+@pytest.mark.parametrize("group", [2, 4, 8])
 def test_gqa_fused_append(group):
     kv_heads = 2
     lens = [3, 16, 17, 600, 1, 2048]

@@ -33,7 +33,7 @@ PS = 64  # several partitions per long sequence, so merges run
 
 
 def _case(group):
-    """Group 1 runs the CUDA-core kernel, group 4 the tensor-core one."""
+    """Group 1 runs the CUDA-core kernel, groups 2 and 4 the tensor-core one."""
     H = 4
     case = syn.decode_case(7, LENS, heads=H, head_dim=128, dtype=np.float16)
     rng = np.random.default_rng(8)
@@ -68,7 +68,7 @@ def _replan_and_check(case, t, ref):
     assert_parity(out, ref, "after a new plan")
 
 
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4])
 def test_a_workspace_that_lost_its_plan_is_refused(group):
     case, t, ref = _case(group)
     _plan(case, t)
@@ -81,7 +81,7 @@ def test_a_workspace_that_lost_its_plan_is_refused(group):
     _replan_and_check(case, t, ref)
 
 
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4])
 @pytest.mark.parametrize("byte", [0x7F, 0xFF])
 def test_damaged_plan_entries_are_skipped(group, byte):
     """Header intact, every per-sequence entry replaced: 0x7f7f7f7f and -1
@@ -96,7 +96,7 @@ def test_damaged_plan_entries_are_skipped(group, byte):
     _replan_and_check(case, t, ref)
 
 
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4])
 def test_random_plan_entries_stay_in_bounds(group):
     """Header intact, the rest random: whatever entries pass the checks index
     only inside the caller's buffers (the result is then meaningless, which
@@ -115,7 +115,7 @@ def test_random_plan_entries_stay_in_bounds(group):
     _replan_and_check(case, t, ref)
 
 
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4])
 def test_a_poisoned_plan_is_refused_until_rewritten(group):
     """A launch that gives up on a wait marks its plan, since the merge
     counters may then be stale.  Set the mark by hand: the next launch on the

@@ -284,7 +284,7 @@ def test_shared_prefix_path_on_the_forked_prompt():
     assert_parity(out, g["out"].double().cpu().numpy(), "shared-prefix vs plain path")
 
 
-@pytest.mark.parametrize("dtype,group", [("f16", 1), ("bf16", 4), ("f16", 8)])
+@pytest.mark.parametrize("dtype,group", [("f16", 1), ("bf16", 2), ("bf16", 4), ("f16", 8)])
 def test_shared_prefix_groups_with_gqa_and_a_bad_member(dtype, group):
     rng = np.random.default_rng(60 + group)
     H, D = 2, 128
@@ -337,7 +337,7 @@ def test_shared_prefix_groups_with_gqa_and_a_bad_member(dtype, group):
     assert_parity(out, ref, f"shared prefix {dtype} G={group}")
 
 
-@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("group", [1, 2, 4])
 def test_shared_prefix_partials_are_read_after_their_kernel(group):
     """The decode launch may overlap the shared-prefix kernel before it and
     reads that kernel's partials only once it has completed.  A long shared
