@@ -190,6 +190,9 @@ __global__ void __launch_bounds__(128)
   const int HK = a.heads, HQ = a.heads * G;
   const int PS = a.partition_size;
 
+  // launched right behind its plan (one call that plans and runs): the CTAs
+  // set up while the plan kernel runs, and wait for it here
+  if (a.after_plan) grid_dependency_wait();
   int32_t next = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);

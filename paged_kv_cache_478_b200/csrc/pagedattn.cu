@@ -214,9 +214,10 @@ cudaError_t set_gqa_attrs() {
 }
 
 // Launch a persistent decode kernel.  With `overlap`, it is a programmatic
-// dependent launch on the preceding kernel of the stream (the shared-prefix
-// kernel): its CTAs may start while that kernel runs, and wait for it only
-// before merging a sequence that has shared-prefix partials.
+// dependent launch on the preceding kernel of the stream: the shared-prefix
+// kernel (the decode CTAs wait for it only before merging a sequence that
+// has shared-prefix partials) or the plan kernel (a.after_plan: they wait for
+// it before reading the plan).
 template <typename K, typename... Extra>
 cudaError_t launch_decode_grid(K kernel, int grid, int threads, size_t smem, cudaStream_t stream,
                                const DecodeArgs& a, bool overlap, const Extra&... extra) {
@@ -791,7 +792,8 @@ pa_status pa_decode_attention(const pa_pool* pool, const void* q, const void* k_
   set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = launch_plan(pool, &a, s)) != PA_OK) return st;
-  return launch_run(pool, a, *dev, s);
+  a.after_plan = 1;  // the decode launch overlaps the plan kernel's run
+  return launch_run(pool, a, *dev, s, true);
 }
 
 pa_status pa_decode_append_attention_planned(const pa_pool* pool, const void* q,
@@ -831,14 +833,25 @@ pa_status pa_decode_append_attention(const pa_pool* pool, const void* q, const v
   CallRange range("pa_decode_append_attention");
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode append: num_seqs < 0");
   if (num_seqs == 0) return check_pool(pool);
-  pa_status st = pa_decode_plan(pool, context_lens, num_seqs, max_blocks_per_seq,
-                                max_context_len, partition_size, workspace, workspace_bytes,
-                                stream);
+  pa_status st = check_run_pointers(q, k_pool, v_pool, block_tables, out, scale);
   if (st != PA_OK) return st;
-  return pa_decode_append_attention_planned(pool, q, k_new, v_new, k_pool, v_pool, block_tables,
-                                            max_blocks_per_seq, num_seqs, max_context_len, scale,
-                                            out, workspace, workspace_bytes, partition_size,
-                                            stream);
+  if (!context_lens) return fail(PA_ERR_INVALID_ARG, "decode append: context_lens is null");
+  if (!k_new || !v_new) return fail(PA_ERR_INVALID_ARG, "decode append: k_new/v_new is null");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(PA_ERR_INVALID_ARG, "decode append: k_new/v_new must be 16-byte aligned");
+  DecodeArgs a;
+  DeviceState* dev;
+  st = prepare_decode(pool, num_seqs, max_blocks_per_seq, max_context_len, partition_size,
+                      workspace, workspace_bytes, &a, &dev);
+  if (st != PA_OK) return st;
+  a.context_lens = context_lens;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = launch_plan(pool, &a, s)) != PA_OK) return st;
+  set_run_args(&a, q, k_pool, v_pool, block_tables, out, scale);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.after_plan = 1;  // the decode launch overlaps the plan kernel's run
+  return launch_run(pool, a, *dev, s, true);
 }
 
 pa_status pa_decode_attention_shared_prefix(

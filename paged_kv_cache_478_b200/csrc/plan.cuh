@@ -72,6 +72,7 @@ struct DecodeArgs {
   int32_t max_context_len;
   float scale_log2;  // scale * log2(e)
   uint64_t stamp;    // number of the plan the host expects in the workspace
+  int32_t after_plan;  // launched as a programmatic dependent of the plan kernel: wait for it first
 };
 
 // Checks a CTA makes before it trusts the plan in the workspace: the header
@@ -112,6 +113,9 @@ __device__ __forceinline__ bool plan_item(const DecodeArgs& a, int item, PlanIte
 // ---- plan: one CTA orders the work ------------------------------------------------
 
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeArgs a) {
+  // a decode launch that follows as a programmatic dependent may start its
+  // CTAs now; they wait for this grid to complete before reading the plan
+  grid_dependents_launch();
   // bucket[0..nb]: ragged last partitions of split sequences by block count;
   // bucket[nb+1..2nb+1]: unsplit sequences by block count (nb+1: no own tokens)
   extern __shared__ int32_t bucket[];
