@@ -106,7 +106,8 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
   // the max over the partitions while the first round flies: the head's LPH
   // lanes read every LPH-th partition, then combine (max is exact)
   float M = -INFINITY;
-  for (int p = lane % LPH; p < np; p += LPH) M = fmaxf(M, __ldcg(&ml[p]).x);
+#pragma unroll 4
+  for (int p = lane % LPH; p < np; p += LPH) M = fmaxf(M, __ldcg(&ml[p]).x);  // loads in flight together
 #pragma unroll
   for (int m = 1; m < LPH; m <<= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
 
