@@ -60,7 +60,12 @@ struct GqaConfig {
 
 // Merge the partitions of all G query heads of one KV head (query heads
 // sh0 .. sh0+G-1) with one warp: 32/G lanes per query head, each lane owning
-// D*G/32 output dimensions, so the G merges run side by side.  The partial
+// D*G/32 output dimensions, so the G merges run side by side.  A lane owns
+// every (32/G)-th 16-byte chunk of its head's row, so that one load
+// instruction of the warp reads whole 128-byte lines of the staged rows; with
+// 8 heads (64 bytes per head and instruction) the odd heads take their
+// chunks in the opposite order of each pair, so that the 8 heads fill all 32
+// banks and no two lanes meet in one.  The partial
 // rows are staged through the warp's ring buffer `buf` by bulk copies, PC
 // partitions of every head per round (one copy per head and round, all in
 // flight at once), and the (m, l) pairs of a round are loaded while the
@@ -73,16 +78,19 @@ struct GqaConfig {
 template <typename T, int D, int G, int NSTAGE, int BUF>
 __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, int np, int lane,
                                             uint8_t* buf, uint64_t* bars, uint32_t& fills) {
-  using C = Chunk<T>;
   constexpr int LPH = 32 / G;        // lanes per query head
   constexpr int DPL = D / LPH;       // output dimensions per lane
   constexpr int ROW = D * 4;         // one partial row, fp32
   constexpr int PC = BUF / (G * ROW);  // partitions per round
-  static_assert(DPL % C::N == 0 || DPL == 4, "a lane owns whole 16-byte output chunks");
+  constexpr int CPL = DPL / 4;        // 16-byte chunks per lane
+  static_assert(DPL % 4 == 0, "a lane owns whole 16-byte chunks");
   static_assert(PC >= 1, "the ring holds one partition of every head");
+  static_assert(LPH * 16 >= 64 && (LPH * 16 >= 128 || CPL % 2 == 0), "bank layout of the staged rows");
   const int j = lane / LPH;
   const int64_t sh = sh0 + j;
-  const int d0 = (lane % LPH) * DPL;
+  // chunk of acc[4e .. 4e+3]: cl + LPH * (e ^ flip)
+  const int cl = lane % LPH;
+  const int flip = LPH * 16 < 128 ? (j & 1) : 0;
   const float2* ml = a.part_ml + sh * a.max_parts;
 
   // one round: lane 0 copies partitions [p0, p0 + n) of every head into buf
@@ -134,14 +142,14 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
       if (p < n) {
         const float w = exp2f(v[p].x - M);
         den = fmaf(v[p].y, w, den);
-        const float4* src = reinterpret_cast<const float4*>(buf + (j * PC + p) * ROW + d0 * 4);
+        const float4* src = reinterpret_cast<const float4*>(buf + (j * PC + p) * ROW) + cl;
 #pragma unroll
-        for (int e = 0; e < DPL; e += 4) {
-          const float4 x = src[e / 4];
-          acc[e] = fmaf(w, x.x, acc[e]);
-          acc[e + 1] = fmaf(w, x.y, acc[e + 1]);
-          acc[e + 2] = fmaf(w, x.z, acc[e + 2]);
-          acc[e + 3] = fmaf(w, x.w, acc[e + 3]);
+        for (int e = 0; e < CPL; ++e) {
+          const float4 x = src[LPH * (e ^ flip)];
+          acc[4 * e] = fmaf(w, x.x, acc[4 * e]);
+          acc[4 * e + 1] = fmaf(w, x.y, acc[4 * e + 1]);
+          acc[4 * e + 2] = fmaf(w, x.z, acc[4 * e + 2]);
+          acc[4 * e + 3] = fmaf(w, x.w, acc[4 * e + 3]);
         }
       }
     }
@@ -153,13 +161,11 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
   const float inv = 1.f / den;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] *= inv;
-  if constexpr (DPL % C::N == 0) {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + sh * D + d0);
+  uint2* dst = reinterpret_cast<uint2*>(static_cast<T*>(a.out) + sh * D) + cl;
 #pragma unroll
-    for (int c = 0; c < DPL / C::N; ++c) dst[c] = C::from_float(acc + c * C::N);
-  } else {
-    store_out<T, DPL>(static_cast<T*>(a.out) + sh * D + d0, acc);
-  }
+  for (int e = 0; e < CPL; ++e)
+    dst[LPH * (e ^ flip)] = make_uint2(MmaType<T>::pack(acc[4 * e], acc[4 * e + 1]),
+                                       MmaType<T>::pack(acc[4 * e + 2], acc[4 * e + 3]));
   __syncwarp();  // buf is read before the ring's next fill
   return true;
 }
