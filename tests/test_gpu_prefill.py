@@ -18,7 +18,7 @@ from tests.gpu_cases import assert_parity, dev
 pytestmark = pytest.mark.gpu
 
 
-def _case(seed, ctx_new, kv_heads, group, head_dim, dtype):
+def _case(seed, ctx_new, kv_heads, group, head_dim, dtype, wide_v=0):
     rng = np.random.default_rng(seed)
     S = len(ctx_new)
     lens = np.array([c for c, _ in ctx_new], dtype=np.int32)
@@ -35,6 +35,9 @@ def _case(seed, ctx_new, kv_heads, group, head_dim, dtype):
     shape = (nb, kv_heads, 16, head_dim)
     kf = rng.standard_normal(shape).astype(np.float32)
     vf = rng.standard_normal(shape).astype(np.float32)
+    if wide_v:  # values an fp16 V cannot hold, at random places
+        at = tuple(rng.integers(0, n, wide_v) for n in shape)
+        vf[at] = rng.choice([-1.0, 1.0], wide_v) * rng.uniform(7.0e4, 3.0e5, wide_v)
     T = int(news.sum())
     qf = rng.standard_normal((T, kv_heads * group, head_dim)).astype(np.float32)
     qs = np.concatenate([[0], np.cumsum(news)]).astype(np.int32)
@@ -202,3 +205,18 @@ def test_prefill_with_several_items_per_cta(kv_heads, group):
     ref = oracle.decode_attention(qt.numpy()[rows], kt.numpy(), vt.numpy(), np.stack(row_t),
                                   np.array(row_l, np.int32), scale)
     assert_parity(out[rows], ref, f"prefill, several items per CTA, G={group}")
+
+
+@pytest.mark.parametrize("head_dim,group", [(128, 1), (64, 4)])
+def test_prefill_bf16_keeps_v_values_beyond_fp16_range(head_dim, group):
+    """bf16 pools hold values no fp16 operand could (|v| up to 3e5 here, at
+    random places in many tiles): the products stay in bf16 (P as a high part
+    plus residual), so the result matches the oracle and stays finite."""
+    c = _case(91 + group, CASES, 2, group, head_dim, "bf16", wide_v=60)
+    out = torch.empty_like(c["q"])
+    pa.pa_prefill_attention(c["pool"], c["q"], c["k"], c["v"], c["tables"], c["lens"], c["qs"],
+                            c["scale"], out, c["max_new"])
+    assert pa.pa_device_errors() == 0
+    assert torch.isfinite(out.float()).all()
+    assert float(np.abs(c["ref"]).max()) > 100.0  # the wide values reach the outputs
+    assert_parity(out, c["ref"], f"prefill bf16 wide V D={head_dim} G={group}")
