@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   // launched right behind its plan (one call that plans and runs): the CTAs
   // set up while the plan kernel runs, and wait for it here
   if (a.after_plan) grid_dependency_wait();
-  int32_t next = 0;
+  int32_t next = -1;  // thread 0: the next item, once reserved
   if (threadIdx.x == 0) {
     for (int i = 0; i < RINGS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
@@ -301,9 +301,9 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
   uint64_t* my_bars = bars + ring * NSTAGE;
 
   for (;;) {
-    if (threadIdx.x == 0) {
-      s_item = next;
-      if (next < num_items) next = atomicAdd(&a.plan->work_counter, 1);  // prefetch the next index
+    if (threadIdx.x == 0) {  // reserved near the end of the previous item, else taken now
+      s_item = next >= 0 ? next : atomicAdd(&a.plan->work_counter, 1);
+      next = -1;
     }
     __syncthreads();
     const int item = s_item;
@@ -445,6 +445,12 @@ __global__ void __launch_bounds__(WARPS * 32) paged_decode_kernel(DecodeArgs a) 
           fence_proxy_async_shared();
           issue(k + NSTAGE, i + NSTAGE);
         }
+        // The next item is reserved four tiles before this one ends: late enough
+        // that the queue's last items go to the CTAs that free up first (an
+        // item reserved at the start of the current one waited out all of
+        // it, and CTAs that drew the end of the queue sat idle meanwhile),
+        // early enough that the atomic's round trip is hidden.
+        if (threadIdx.x == 0 && i == max(nblk - 5, 0)) next = atomicAdd(&a.plan->work_counter, 1);
       }
       if (!ok) {
         // give up on this item: report, let the copies already issued land,

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(128)
   // launched right behind its plan (one call that plans and runs): the CTAs
   // set up while the plan kernel runs, and wait for it here
   if (a.after_plan) grid_dependency_wait();
-  int32_t next = 0;
+  int32_t next = -1;  // thread 0: the next item, once reserved
   if (threadIdx.x == 0) {
     for (int i = 0; i < WARPS * NSTAGE; ++i) mbar_init(smem_addr(&bars[i]), 1);
     mbar_init_fence();
@@ -221,9 +221,9 @@ __global__ void __launch_bounds__(128)
   const bool row_ok = qrow < G;  // rows 8..15 are never used (G <= 8)
 
   for (;;) {
-    if (threadIdx.x == 0) {
-      s_item = next;
-      if (next < num_items) next = atomicAdd(&a.plan->work_counter, 1);
+    if (threadIdx.x == 0) {  // reserved near the end of the previous item, else taken now
+      s_item = next >= 0 ? next : atomicAdd(&a.plan->work_counter, 1);
+      next = -1;
     }
     __syncthreads();
     const int item = s_item;
@@ -413,6 +413,8 @@ __global__ void __launch_bounds__(128)
         }
         __syncwarp();  // every lane is done with this stage
         if (lane == 0 && i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
+        // as in the MHA kernel: the next item is reserved four tiles before this one ends
+        if (threadIdx.x == 0 && i == max(nblk - 5, 0)) next = atomicAdd(&a.plan->work_counter, 1);
       }
       if (!ok) {
         if (lane == 0) {  // as in the MHA kernel: report, stop, and poison the plan
