@@ -3,8 +3,9 @@
 // With G query heads per KV head, each staged (block, KV head) tile serves G
 // queries: per 16-token block that is a [G x D] . [D x 16] score product and
 // a [G x 16] . [16 x D] value product, i.e. two m16n8k16 chains with the G
-// query heads as the rows.  One warp owns one KV head of the work item and
-// all of its query heads, so the CUDA-core cost per byte no longer grows
+// query heads as the rows.  Two warps own one KV head of the work item and
+// all of its query heads (each half of the partition's blocks, states
+// combined at the end), so the CUDA-core cost per byte no longer grows
 // with G.  With bf16 the softmax weights enter P.V as a high part plus its
 // rounding residual (8 significand bits alone would cost the result
 // precision); fp16 weights go in as they are.  The running max only moves,
@@ -41,8 +42,9 @@ namespace pa {
 
 template <typename T, int D, int NSTAGE>
 struct GqaConfig {
-  static constexpr int WARPS = PA_GQA_WARPS;  // KV heads per work item, one per warp
-  static_assert(WARPS >= 1 && WARPS <= 4, "warps per CTA");
+  static constexpr int WARPS = PA_GQA_WARPS;  // warps per CTA, two per KV head of the work item
+  static_assert(WARPS == 2 || WARPS == 4, "warps per CTA");
+  static constexpr int KVPI = WARPS / 2;      // KV heads per work item
   static constexpr int THREADS = WARPS * 32;
   static constexpr int ROW_BYTES = D * 2;
   static constexpr int BOXES = D / 64;              // 64-wide slices of head_dim
@@ -173,7 +175,7 @@ __device__ __forceinline__ bool merge_group(const DecodeArgs& a, int64_t sh0, in
 // tm_k, tm_v: the K and V pools as [num_blocks * heads * 16 rows][head_dim],
 // box {64, 16}, 128-byte swizzle.
 template <typename T, int D, int NSTAGE>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 3)  // 3 CTAs per SM: at most 168 registers a thread
     paged_decode_gqa_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v) {
   using Cfg = GqaConfig<T, D, NSTAGE>;
@@ -255,7 +257,20 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();
 
-    const int kvh = g * WARPS + warp;
+    // Two warps per KV head: warp 2h streams the first half of the
+    // partition's blocks, warp 2h + 1 the second half, and their softmax
+    // states are combined below.  An item then carries the bytes of two KV
+    // heads, not four, so the queue's items are half as long and the CTAs
+    // finish closer together.
+    const int kvh = g * Cfg::KVPI + (warp >> 1);
+    const int half = warp & 1;
+    const int n0 = (nblk + 1) >> 1;
+    const int jb = half ? n0 : 0;            // this warp's first block of the partition
+    const int my_n = half ? nblk - n0 : n0;  // and its number of blocks
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
     if (kvh < HK) {
       // Q fragments of this KV head's query heads (rows >= G are zero)
       uint32_t qa[KSTEPS][4];
@@ -270,11 +285,6 @@ __global__ void __launch_bounds__(128)
           qa[ks][3] = 0u;
         }
       }
-      float m_run = -INFINITY, l_run = 0.f;
-      float o[NT][2];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
-
       char* kbase = static_cast<char*>(const_cast<void*>(a.k_pool)) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
       char* vbase = static_cast<char*>(const_cast<void*>(a.v_pool)) + (int64_t)kvh * kBlock * Cfg::ROW_BYTES;
       const int64_t block_bytes = (int64_t)HK * kBlock * Cfg::ROW_BYTES;
@@ -297,10 +307,10 @@ __global__ void __launch_bounds__(128)
       const uint32_t k0 = fills;
       __syncwarp();  // every lane is done with the previous item's stages
       if (lane == 0)
-        for (int j = 0; j < NSTAGE && j < nblk; ++j) issue(k0 + j, j);
+        for (int j = 0; j < NSTAGE && j < my_n; ++j) issue(k0 + j, jb + j);
       bool ok = true;
       int i = 0;
-      for (; i < nblk; ++i) {
+      for (; i < my_n; ++i) {
         const uint32_t k = k0 + i;
         const int st = k % NSTAGE;
         const bool landed = mbar_wait_bounded(smem_addr(&my_bars[st]), (k / NSTAGE) & 1u);
@@ -310,7 +320,7 @@ __global__ void __launch_bounds__(128)
         }
         uint8_t* ktile = my_stages + st * Cfg::STAGE_BYTES;
         uint8_t* vtile = ktile + Cfg::TILE_BYTES;
-        const int valid = min(kBlock, ntok - i * kBlock);
+        const int valid = min(kBlock, ntok - (jb + i) * kBlock);
         if (valid < kBlock) {
           // V rows past the context hold stale values (maybe NaN): zero them
           // so that 0-weight x stale never reaches P.V
@@ -321,7 +331,7 @@ __global__ void __launch_bounds__(128)
                                       (c % 8) * 16) = make_uint4(0, 0, 0, 0);
           }
         }
-        if (append && i == nblk - 1 && lane < Cfg::ROW_BYTES / 16) {
+        if (append && jb + i == nblk - 1 && lane < Cfg::ROW_BYTES / 16) {
           // fused reshape_and_cache of the KV head's new row: into the pool,
           // and over the stale row of the staged tiles
           const int64_t skv = (int64_t)s * HK + kvh;
@@ -330,7 +340,7 @@ __global__ void __launch_bounds__(128)
           const uint32_t off = (lane / 8) * Cfg::BOX_BYTES + sw128_off(new_row, lane % 8);
           *reinterpret_cast<uint4*>(ktile + off) = kn;
           *reinterpret_cast<uint4*>(vtile + off) = vn;
-          const int64_t row_off = (int64_t)tbl[i] * block_bytes + (int64_t)new_row * Cfg::ROW_BYTES;
+          const int64_t row_off = (int64_t)tbl[jb + i] * block_bytes + (int64_t)new_row * Cfg::ROW_BYTES;
           reinterpret_cast<uint4*>(kbase + row_off)[lane] = kn;
           reinterpret_cast<uint4*>(vbase + row_off)[lane] = vn;
         }
@@ -412,9 +422,9 @@ __global__ void __launch_bounds__(128)
           }
         }
         __syncwarp();  // every lane is done with this stage
-        if (lane == 0 && i + NSTAGE < nblk) issue(k + NSTAGE, i + NSTAGE);
-        // as in the MHA kernel: the next item is reserved four tiles before this one ends
-        if (threadIdx.x == 0 && i == max(nblk - 5, 0)) next = atomicAdd(&a.plan->work_counter, 1);
+        if (lane == 0 && i + NSTAGE < my_n) issue(k + NSTAGE, jb + i + NSTAGE);
+        // as in the MHA kernel: the next item is reserved a few tiles before this one ends
+        if (threadIdx.x == 0 && i == max(my_n - 3, 0)) next = atomicAdd(&a.plan->work_counter, 1);
       }
       if (!ok) {
         if (lane == 0) {  // as in the MHA kernel: report, stop, and poison the plan
@@ -423,13 +433,44 @@ __global__ void __launch_bounds__(128)
           a.plan->poisoned = 1;
           __threadfence();
         }
-        const int issued = min(nblk, i + NSTAGE);
+        const int issued = min(my_n, i + NSTAGE);
         for (int j = i; j < issued; ++j) {
           const uint32_t k = k0 + j;
           mbar_wait_bounded(smem_addr(&my_bars[k % NSTAGE]), (k / NSTAGE) & 1u);
         }
       } else {
-        fills = k0 + nblk;
+        fills = k0 + my_n;
+        if (half) {  // this half's state, for the other warp of the KV head (its stages are drained)
+          float* xs = reinterpret_cast<float*>(my_stages);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            xs[(2 * j) * 32 + lane] = o[j][0];
+            xs[(2 * j + 1) * 32 + lane] = o[j][1];
+          }
+          xs[2 * NT * 32 + lane] = m_run;
+          xs[(2 * NT + 1) * 32 + lane] = l_run;
+          fence_proxy_async_shared();  // before the ring's next bulk copies into the same bytes
+        }
+      }
+    }
+    __syncthreads();  // both halves of every KV head are done
+    if (kvh < HK && half == 0 && !s_abort) {
+      {  // fold in the second half (log-sum-exp rescale of both to the larger reference max)
+        const float* xs = reinterpret_cast<const float*>(my_stages + NSTAGE * Cfg::STAGE_BYTES);
+        const float mb = xs[2 * NT * 32 + lane], lb = xs[(2 * NT + 1) * 32 + lane];
+        const float M = fmaxf(m_run, mb);
+        const float sa = m_run == -INFINITY ? 0.f : exp2f(m_run - M);
+        const float sb = mb == -INFINITY ? 0.f : exp2f(mb - M);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          o[j][0] = o[j][0] * sa + xs[(2 * j) * 32 + lane] * sb;
+          o[j][1] = o[j][1] * sa + xs[(2 * j + 1) * 32 + lane] * sb;
+        }
+        l_run = l_run * sa + lb * sb;
+        m_run = M;
+        fence_proxy_async_shared();  // the other warp's ring is refilled after the loop's barrier
+      }
+      {
         if (row_ok) {
           const int64_t sh = (int64_t)s * HQ + kvh * G + qrow;
           const int d0 = (lane & 3) * 2;
@@ -461,7 +502,7 @@ __global__ void __launch_bounds__(128)
         if (arrived == ni) *cnt = 0;
       }
       __syncthreads();
-      if (s_merge && kvh < HK) {
+      if (s_merge && kvh < HK && half == 0) {
         if (np > ni) grid_dependency_wait();  // shared-prefix partials: see the MHA kernel
         __threadfence();
         constexpr int BUF = NSTAGE * Cfg::STAGE_BYTES;

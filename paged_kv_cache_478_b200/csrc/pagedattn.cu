@@ -116,7 +116,7 @@ cudaError_t set_decode_attrs_all_groups() {
 int rings_for(int G) { return warps_for(G) / G; }
 
 // Groups of 2, 4 or 8 query heads on fp16/bf16 pools take the tensor-core
-// kernel (one warp per KV head); MHA and fp32 pools take the CUDA-core
+// kernel (two warps per KV head); MHA and fp32 pools take the CUDA-core
 // kernel.  (Pairs once ran faster on CUDA cores; since the tensor-core
 // kernel stages whole tiles and merges all heads of a KV head at once it
 // is faster for them too: 106 -> 89 us on 200 requests x 8 KV heads.)
@@ -127,7 +127,7 @@ bool use_gqa_mma(const pa_pool* pool) { return pool->q_per_kv >= 2 && pool->dtyp
 constexpr int kGqaStages = PA_GQA_STAGES;  // per-warp ring depth of the tensor-core kernel
 
 int kv_heads_per_item(const pa_pool* pool) {
-  return use_gqa_mma(pool) ? GqaConfig<__half, 128, kGqaStages>::WARPS : rings_for(pool->q_per_kv);
+  return use_gqa_mma(pool) ? GqaConfig<__half, 128, kGqaStages>::KVPI : rings_for(pool->q_per_kv);
 }
 
 template <typename T, int D>
