@@ -140,9 +140,11 @@ pa_status pa_decode_workspace_bytes(const pa_pool* pool, int32_t num_seqs,
  * multiple of 16 up to 4096) whose partial results are merged by
  * log-sum-exp, in partition order, by the last CTA to finish a sequence.
  * partition_size 0 chooses automatically: 512-token partitions while
- * sequences x head groups already give two work items per resident CTA,
- * otherwise about four items per resident CTA (never below 256 tokens).  The work order is planned on the device
- * from context_lens (longest partitions first).
+ * sequences x head groups already give two work items per resident CTA
+ * (one with 2-8 query heads per KV head on fp16/bf16 pools), otherwise
+ * about four items per resident CTA (never below 256 tokens).  The work
+ * order is planned on the device from context_lens (longest partitions
+ * first).
  * max_context_len bounds every context_lens[s] (0 = max_blocks_per_seq *
  * block_size); a length above it or above the table width sets
  * PA_DEVERR_CONTEXT_LEN and is clamped.  Block ids outside the pool set

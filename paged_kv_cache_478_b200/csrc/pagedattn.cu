@@ -373,12 +373,15 @@ int round_up16(int64_t x) { return (int)std::min<int64_t>(kMaxPartition, (x + 15
 // split costs partial results and a merge, while one long item is streamed
 // by a single CTA at a fraction of the chip's bandwidth and can become the
 // critical path.  Measured on B200: when (sequences x head groups) already
-// gives two items per resident CTA, 512-token partitions are best; with few
-// sequences, aim for about four items per resident CTA (never below 256).
-int auto_partition(int num_seqs, int head_groups, int max_context_len, int slots) {
+// gives `full_items` items per resident CTA, 512-token partitions are best
+// (2 for the CUDA-core kernel; 1 for the tensor-core GQA kernel, whose items
+// of 2 KV heads are streamed by 4 warps: 200 requests x 8 KV heads took
+// 84.7 us at 512 tokens against 88.5 at the 352 the rule below gives); with
+// few sequences, aim for about four items per resident CTA (never below 256).
+int auto_partition(int num_seqs, int head_groups, int max_context_len, int slots, int full_items) {
   const int64_t whole = (int64_t)num_seqs * head_groups;
   const int64_t maxL = std::max(16, max_context_len);
-  if (whole >= 2LL * slots) return std::min(kFullBatchPartition, round_up16(maxL));
+  if (whole >= (int64_t)full_items * slots) return std::min(kFullBatchPartition, round_up16(maxL));
   // About 4 work items per resident CTA.  Only the longest context is known
   // here; a ragged batch averages about half of it, so the partitions are
   // sized for maxL / 2 (sizing them for maxL left items too long to balance).
@@ -560,7 +563,8 @@ pa_status prepare_decode(const pa_pool* pool, int32_t num_seqs, int32_t max_bloc
                  : max_shared_blocks > 0
                      ? kMinAutoPartition
                      : auto_partition(num_seqs, head_groups, maxL,
-                                      (*dev)->num_sms * (*dev)->decode_ctas_per_sm);
+                                      (*dev)->num_sms * (*dev)->decode_ctas_per_sm,
+                                      use_gqa_mma(pool) ? 1 : 2);
   const int max_parts = total_parts(maxL, ps, max_shared_blocks);
   const WorkspaceLayout w = layout_for(num_seqs, (int64_t)pool->heads * G, max_parts,
                                        pool->head_dim, G, kv_heads_per_item(pool));
