@@ -253,7 +253,7 @@ def long_context(partition_size: int = 0, profile: bool = False):
                       "us": round(ms * 1e3, 1), "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
 
-def single_layer(profile: bool = False):
+def single_layer(partition_size: int = 0, profile: bool = False):
     """One layer of 64 sequences, lengths uniform in [1, 2048], 32 heads x 128
     fp16, the pool exactly the used blocks at random places; the new token is
     appended and attended in one launch (about 1.1 GB of K/V, larger than L2)."""
@@ -268,11 +268,11 @@ def single_layer(profile: bool = False):
     kn, vn = torch.randn_like(q), torch.randn_like(q)
     pool = pa.pa_pool_create(nb, 16, H, D, torch.float16)
     bt, cl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
-    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1]), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(pa.pa_decode_workspace_bytes(pool, S, tables.shape[1], 0, partition_size),
+                     dtype=torch.uint8, device="cuda")
     out = torch.empty_like(q)
     run = lambda: pa.pa_decode_append_attention(  # noqa: E731
-        pool, q, kn, vn, kp, vp, bt, cl, 1 / math.sqrt(D), out, ws)
+        pool, q, kn, vn, kp, vp, bt, cl, 1 / math.sqrt(D), out, ws, partition_size=partition_size)
     if profile:
         _profile_launches(run, "single layer: 64 sequences, plan + append + attend")
         return
@@ -280,6 +280,7 @@ def single_layer(profile: bool = False):
     _check()
     kv_bytes = int(lens.sum()) * H * D * 2 * 2
     print(json.dumps({"kernel": "decode (single layer, plan + append + attend)", "sequences": S,
+                      "partition_size": partition_size or "auto",
                       "cached_tokens": int(lens.sum()), "us": round(ms * 1e3, 1),
                       "kv_GBps": round(kv_bytes / ms / 1e6, 1)}))
 
@@ -372,6 +373,7 @@ def main(argv=None):
     p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     p.add_argument("--profile", action="store_true")
     p = sub.add_parser("single-layer")
+    p.add_argument("--partition-size", type=int, default=0, help="0 = automatic")
     p.add_argument("--profile", action="store_true")
     p = sub.add_parser("cache-ops")
     p.add_argument("--profile", action="store_true")
@@ -390,7 +392,7 @@ def main(argv=None):
     elif args.what == "long-context":
         long_context(args.partition_size, args.profile)
     elif args.what == "single-layer":
-        single_layer(args.profile)
+        single_layer(args.partition_size, args.profile)
     elif args.what == "cache-ops":
         cache_ops(args.profile)
     else:
