@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(128, 3)  // 3 CTAs per SM: at most 168 registe
     // Two warps per KV head: warp 2h streams the first half of the
     // partition's blocks, warp 2h + 1 the second half, and their softmax
     // states are combined below.  An item then carries the bytes of two KV
-    // heads, not four, so the queue's items are half as long and the CTAs
-    // finish closer together.
+    // heads, not four: at a given partition size the queue's items are half
+    // as long, which makes longer partitions (fewer merges) affordable.
     const int kvh = g * Cfg::KVPI + (warp >> 1);
     const int half = warp & 1;
     const int n0 = (nblk + 1) >> 1;
@@ -470,24 +470,22 @@ __global__ void __launch_bounds__(128, 3)  // 3 CTAs per SM: at most 168 registe
         m_run = M;
         fence_proxy_async_shared();  // the other warp's ring is refilled after the loop's barrier
       }
-      {
-        if (row_ok) {
-          const int64_t sh = (int64_t)s * HQ + kvh * G + qrow;
-          const int d0 = (lane & 3) * 2;
-          if (!split) {
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            T* dst = static_cast<T*>(a.out) + sh * D + d0;
+      if (row_ok) {  // the output rows, or the partition's partials
+        const int64_t sh = (int64_t)s * HQ + kvh * G + qrow;
+        const int d0 = (lane & 3) * 2;
+        if (!split) {
+          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          T* dst = static_cast<T*>(a.out) + sh * D + d0;
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-              const uint32_t v = MmaType<T>::pack(o[j][0] * inv, o[j][1] * inv);
-              *reinterpret_cast<uint32_t*>(dst + j * 8) = v;
-            }
-          } else {
-            float* dst = a.part_acc + (sh * a.max_parts + p) * D + d0;
-#pragma unroll
-            for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
-            if ((lane & 3) == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
+          for (int j = 0; j < NT; ++j) {
+            const uint32_t v = MmaType<T>::pack(o[j][0] * inv, o[j][1] * inv);
+            *reinterpret_cast<uint32_t*>(dst + j * 8) = v;
           }
+        } else {
+          float* dst = a.part_acc + (sh * a.max_parts + p) * D + d0;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) *reinterpret_cast<float2*>(dst + j * 8) = make_float2(o[j][0], o[j][1]);
+          if ((lane & 3) == 0) a.part_ml[sh * a.max_parts + p] = make_float2(m_run, l_run);
         }
       }
     }
